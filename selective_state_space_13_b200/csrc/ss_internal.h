@@ -1,0 +1,67 @@
+// Internal declarations shared by the host entry points (ss_api.cu) and the kernels (ss_scan.cu).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "selective_scan.h"
+
+namespace ss {
+
+// Steps per pipeline stage and number of stages of the shared-memory ring.
+constexpr int kTile = 32;
+constexpr int kStages = 4;
+
+// Everything a scan launch needs.  Device pointers are the caller's; nothing here is owned.
+struct ScanParams {
+    const void* u;          // [batch, L, D] io, spatial order
+    const void* delta;      // [K, batch, L, D] io, scan order
+    const float* A;         // [D, N]
+    const void* B;          // [K, batch, L, N] io, scan order
+    const void* C;          // [K, batch, L, N] io, scan order
+    const float* Dskip;     // [D] or null
+    const void* z;          // [batch, L, D] io or null
+    const float* bias;      // [D] or null
+    void* out;              // [batch, L, D] io (single direction) or null
+    float* ypart;           // [K, batch, L, D] fp32 per-direction outputs (several directions)
+    float* last_state;      // [K, batch, D, N] or null
+    float* carry_h;         // [K, batch, S, D, N] end state of each segment scanned from zero
+    float* carry_s;         // [K, batch, S, D] sum over the segment of Delta*log2(e)
+    int64_t batch, L, D;
+    int64_t seg_len;        // steps per segment (last segment may be shorter)
+    int32_t N, K, S;
+    int32_t dirs[SS_MAX_DIRS];
+    int32_t H, W;
+    int32_t softplus;
+    int32_t force_generic;  // 1: never take the A[d,n] = (n+1) A[d,0] shortcut
+};
+
+struct MergeParams {
+    const float* ypart;     // [K, batch, L, D]
+    const void* z;          // [batch, L, D] io or null
+    void* out;              // [batch, L, D] io
+    int64_t rows;           // batch * L
+    int64_t D;
+    int32_t K;
+};
+
+// Channels handled by one CTA of the scan kernel (one thread per channel).
+int channels_per_cta();
+
+// Enqueue one scan launch.  phase1 = 1: segment aggregates only (segments 0..S-2);
+// phase1 = 0: full scan of all S segments.  Returns the CUDA error of the launch.
+cudaError_t launch_scan(const ScanParams& p, int io_dtype, int phase1, cudaStream_t stream);
+
+// Enqueue the direction merge + gate: out = (sum_k ypart[k]) * silu(z).
+cudaError_t launch_merge(const MergeParams& p, int io_dtype, cudaStream_t stream);
+
+// Same index function the kernels use (host copy of the device function).
+int64_t position_host(int32_t dir, int64_t L, int32_t H, int32_t W, int64_t t);
+
+// Synchronise `stream`, read this library's device error word on the current device into *value,
+// and reset it when `clear` is set.
+cudaError_t read_status(cudaStream_t stream, bool clear, unsigned int* value);
+
+}  // namespace ss

@@ -1,0 +1,296 @@
+"""Python binding of the C ABI in include/selective_scan.h (argument marshalling only).
+
+Every step of the scan runs in the CUDA library libss_b200.so; this module checks tensor
+shapes, dtypes and devices, allocates outputs and the workspace through PyTorch when the
+caller did not pass them, and calls the library on the current CUDA stream.  There is no CPU
+path: without the library, or without a CUDA device, every call raises.
+
+The functions carry the C names: selective_scan_fwd, selective_scan_workspace_size,
+ss_direction_position, selective_scan_device_status, ss_status_str, ss_abi_version.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import hashlib
+import os
+import threading
+
+from . import build as _build
+
+SS_OK = 0
+SS_F32, SS_BF16 = 0, 1
+SS_DIR_FWD, SS_DIR_REV, SS_DIR_COL, SS_DIR_COL_REV = 0, 1, 2, 3
+SS_FLAG_GENERIC_A = 1
+SS_MAX_DSTATE = 16
+SS_MAX_DIRS = 4
+
+STATUS_NAMES = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE",
+                4: "SS_ERR_ALIGN", 5: "SS_ERR_DIRMAP", 6: "SS_ERR_UNSUPPORTED", 7: "SS_ERR_CUDA",
+                8: "SS_ERR_WORKSPACE", 9: "SS_ERR_DEVICE_TIMEOUT"}
+
+EXPORTED = ("selective_scan_workspace_size", "selective_scan_fwd", "ss_direction_position",
+            "selective_scan_device_status", "ss_status_str", "ss_abi_version")
+
+
+class SsShape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("dim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("io_dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+class SsDirectionMap(ctypes.Structure):
+    _fields_ = [("num_dirs", ctypes.c_int32), ("dir", ctypes.c_int32 * SS_MAX_DIRS),
+                ("H", ctypes.c_int32), ("W", ctypes.c_int32)]
+
+
+class SsLaunchOpts(ctypes.Structure):
+    _fields_ = [("segments", ctypes.c_int32), ("flags", ctypes.c_int32),
+                ("scan_begin_event", ctypes.c_void_p), ("scan_end_event", ctypes.c_void_p),
+                ("reserved", ctypes.c_int32 * 4)]
+
+
+class ScanError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__("%s%s" % (ss_status_str(status), (": " + what) if what else ""))
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def _source_digest() -> str:
+    h = hashlib.sha256()
+    for f in _build.SOURCES + _build.HEADERS:
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def ensure_built() -> str:
+    """Build libss_b200.so when it is missing or its sources changed (by content)."""
+    stamp = _build.LIB + ".srchash"
+    digest = _source_digest()
+    have = None
+    if os.path.exists(_build.LIB) and os.path.exists(stamp):
+        with open(stamp) as fh:
+            have = fh.read().strip()
+    if have != digest:
+        _build.build(force=True)
+        with open(stamp, "w") as fh:
+            fh.write(digest)
+    return _build.LIB
+
+
+def load():
+    """Load the CUDA library (building it first if needed) and declare its signatures."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = ensure_built()
+        lib = ctypes.CDLL(path)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        lib.selective_scan_workspace_size.restype = ctypes.c_int
+        lib.selective_scan_workspace_size.argtypes = [ctypes.POINTER(SsShape),
+                                                      ctypes.POINTER(SsDirectionMap),
+                                                      ctypes.POINTER(SsLaunchOpts),
+                                                      ctypes.POINTER(sz)]
+        lib.selective_scan_fwd.restype = ctypes.c_int
+        lib.selective_scan_fwd.argtypes = [ctypes.POINTER(SsShape), vp, vp, vp, vp, vp, vp, vp, vp,
+                                           i32, ctypes.POINTER(SsDirectionMap), vp, vp, vp, sz, vp,
+                                           ctypes.POINTER(SsLaunchOpts)]
+        lib.ss_direction_position.restype = i64
+        lib.ss_direction_position.argtypes = [ctypes.POINTER(SsDirectionMap), i32, i64, i64]
+        lib.selective_scan_device_status.restype = ctypes.c_int
+        lib.selective_scan_device_status.argtypes = [vp, i32]
+        lib.ss_status_str.restype = ctypes.c_char_p
+        lib.ss_status_str.argtypes = [ctypes.c_int]
+        lib.ss_abi_version.restype = i32
+        lib.ss_abi_version.argtypes = []
+        _lib = lib
+        return lib
+
+
+# ----------------------------------------------------------------------------- thin C wrappers
+
+def ss_status_str(status: int) -> str:
+    try:
+        return load().ss_status_str(int(status)).decode()
+    except OSError:
+        return STATUS_NAMES.get(int(status), "unknown ss_status %d" % status)
+
+
+def ss_abi_version() -> int:
+    return int(load().ss_abi_version())
+
+
+def make_shape(batch, seqlen, dim, dstate, io_dtype) -> SsShape:
+    return SsShape(int(batch), int(seqlen), int(dim), int(dstate), int(io_dtype), 0)
+
+
+def make_dirmap(dirs=(SS_DIR_FWD,), H=0, W=0) -> SsDirectionMap:
+    m = SsDirectionMap()
+    m.num_dirs = len(dirs)
+    for i, d in enumerate(list(dirs)[:SS_MAX_DIRS]):
+        m.dir[i] = int(d)
+    m.H, m.W = int(H), int(W)
+    return m
+
+
+def make_opts(segments=0, flags=0, events=None) -> SsLaunchOpts:
+    """events: optional (begin, end) torch.cuda.Event pair, recorded by the library around its
+    main scan launch on the call's stream (each must have been recorded once before, so that
+    its CUDA event exists)."""
+    o = SsLaunchOpts()
+    o.segments, o.flags = int(segments), int(flags)
+    if events is not None:
+        o.scan_begin_event = int(events[0].cuda_event) or None
+        o.scan_end_event = int(events[1].cuda_event) or None
+    return o
+
+
+def selective_scan_workspace_size(shape: SsShape, dmap: SsDirectionMap | None = None,
+                                  opts: SsLaunchOpts | None = None) -> int:
+    n = ctypes.c_size_t(0)
+    st = load().selective_scan_workspace_size(ctypes.byref(shape),
+                                              ctypes.byref(dmap) if dmap is not None else None,
+                                              ctypes.byref(opts) if opts is not None else None,
+                                              ctypes.byref(n))
+    if st != SS_OK:
+        raise ScanError(st, "selective_scan_workspace_size")
+    return int(n.value)
+
+
+def ss_direction_position(dmap: SsDirectionMap | None, k: int, L: int, t: int) -> int:
+    return int(load().ss_direction_position(ctypes.byref(dmap) if dmap is not None else None,
+                                            int(k), int(L), int(t)))
+
+
+def selective_scan_device_status(stream=None, clear: bool = True) -> int:
+    """Synchronise the stream and return SS_OK or SS_ERR_DEVICE_TIMEOUT (see the C header)."""
+    return int(load().selective_scan_device_status(_stream_handle(stream), int(bool(clear))))
+
+
+def selective_scan_fwd_raw(shape: SsShape, u, delta, A, B, C, Dskip, z, delta_bias, softplus,
+                           dmap, out, last_state, workspace, workspace_bytes, stream,
+                           opts=None) -> int:
+    """Direct call with integer device addresses (0 = NULL); returns the ss_status."""
+    return int(load().selective_scan_fwd(
+        ctypes.byref(shape), u or None, delta or None, A or None, B or None, C or None,
+        Dskip or None, z or None, delta_bias or None, int(bool(softplus)),
+        ctypes.byref(dmap) if dmap is not None else None, out or None, last_state or None,
+        workspace or None, int(workspace_bytes), stream or None,
+        ctypes.byref(opts) if opts is not None else None))
+
+
+# ----------------------------------------------------------------------------- torch front end
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ptr(t):
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _io_code(dtype):
+    import torch
+    if dtype == torch.float32:
+        return SS_F32
+    if dtype == torch.bfloat16:
+        return SS_BF16
+    raise TypeError("io tensors must be float32 or bfloat16, got %s" % dtype)
+
+
+def _check(t, name, shape, dtype, device):
+    if t is None:
+        return
+    if not t.is_cuda or t.device != device:
+        raise ValueError("%s must be a CUDA tensor on %s" % (name, device))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+_ws_cache = {}
+
+
+def _workspace(nbytes, device):
+    import torch
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf
+
+
+def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                       dirs=(SS_DIR_FWD,), H=0, W=0, out=None, last_state=None,
+                       return_last_state=False, workspace=None, stream=None, segments=0,
+                       flags=0, events=None):
+    """Selective scan forward on CUDA tensors.
+
+    u, z: [batch, L, D]; delta: [K, batch, L, D] (or [batch, L, D] when K = 1); B, C:
+    [K, batch, L, N] (or [batch, L, N]); A: [D, N] float32; D (skip) and delta_bias: [D] float32.
+    u, delta, B, C, z share one dtype (float32 or bfloat16); out has that dtype.
+    Returns out, or (out, last_state [K, batch, D, N] float32) with return_last_state.
+    """
+    import torch
+    device = u.device
+    if u.dim() != 3:
+        raise ValueError("u must be [batch, L, D]")
+    batch, L, Dm = u.shape
+    K = len(dirs)
+    if delta.dim() == 3:
+        delta = delta.unsqueeze(0)
+    if B.dim() == 3:
+        B = B.unsqueeze(0)
+    if C.dim() == 3:
+        C = C.unsqueeze(0)
+    N = A.shape[-1]
+    io = u.dtype
+    _io_code(io)
+    _check(u, "u", (batch, L, Dm), io, device)
+    _check(delta, "delta", (K, batch, L, Dm), io, device)
+    _check(B, "B", (K, batch, L, N), io, device)
+    _check(C, "C", (K, batch, L, N), io, device)
+    _check(z, "z", (batch, L, Dm), io, device)
+    _check(A, "A", (Dm, N), torch.float32, device)
+    _check(D, "D", (Dm,), torch.float32, device)
+    _check(delta_bias, "delta_bias", (Dm,), torch.float32, device)
+    if out is None:
+        out = torch.empty_like(u)
+    _check(out, "out", (batch, L, Dm), io, device)
+    if return_last_state and last_state is None:
+        last_state = torch.empty((K, batch, Dm, N), dtype=torch.float32, device=device)
+    _check(last_state, "last_state", (K, batch, Dm, N), torch.float32, device)
+    shape = make_shape(batch, L, Dm, N, _io_code(io))
+    dmap = make_dirmap(dirs, H, W)
+    opts = make_opts(segments, flags, events)
+    nws = selective_scan_workspace_size(shape, dmap, opts)
+    if workspace is None and nws > 0:
+        workspace = _workspace(nws, device)
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = selective_scan_fwd_raw(shape, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                _ptr(z), _ptr(delta_bias), softplus, dmap, _ptr(out),
+                                _ptr(last_state), _ptr(workspace), wsb, _stream_handle(stream),
+                                opts)
+    if st != SS_OK:
+        raise ScanError(st, "selective_scan_fwd")
+    return (out, last_state) if return_last_state else out

@@ -1,0 +1,158 @@
+"""The C ABI on the host, without a GPU: the library loads, exports every symbol the header
+declares, rejects bad arguments with the documented status before touching any device, and its
+index map (the very function the kernels use) matches the oracle's independent one bit for bit."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from selective_state_space_13_b200 import scan
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "selective_scan.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*"
+                                 r"([A-Za-z_][A-Za-z0-9_]*)\s*\(", text, flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = scan.load()
+    names = header_functions()
+    assert set(names) == set(scan.EXPORTED), names
+    for name in names:
+        assert hasattr(lib, name), name
+    assert scan.ss_abi_version() == 1
+
+
+def test_status_strings():
+    for code, name in scan.STATUS_NAMES.items():
+        assert scan.ss_status_str(code).startswith(name)
+
+
+def _shape(**kw):
+    base = dict(batch=2, seqlen=64, dim=32, dstate=16, io_dtype=scan.SS_BF16)
+    base.update(kw)
+    return scan.make_shape(**base)
+
+
+FAKE = 1 << 20  # a 16-byte aligned, never dereferenced address: validation must fail first
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dstate=0), 2),
+    (dict(dstate=17), 6),
+    (dict(batch=-1), 2),
+    (dict(seqlen=1 << 31), 2),
+    (dict(io_dtype=7), 3),
+    (dict(dim=12), 4),            # 12 * 2 bytes is not a multiple of 16
+])
+def test_shape_validation(kw, expect):
+    sh = _shape(**kw)
+    with pytest.raises(scan.ScanError) as ei:
+        scan.selective_scan_workspace_size(sh)
+    assert ei.value.status == expect
+    st = scan.selective_scan_fwd_raw(sh, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, 0, 1, None, FAKE, 0,
+                                     0, 0, 0)
+    assert st == expect
+
+
+@pytest.mark.parametrize("dirs,H,W,expect", [
+    ((), 0, 0, 5), ((0, 1, 2, 3, 0), 8, 8, 5), ((4,), 0, 0, 5), ((2,), 8, 7, 5),
+    ((2,), 0, 64, 5), ((0, 1), 0, 0, 0), ((2, 3), 8, 8, 0), ((3,), 4, 16, 0)])
+def test_dirmap_validation(dirs, H, W, expect):
+    sh = _shape()
+    dm = scan.make_dirmap(dirs, H, W) if dirs else scan.SsDirectionMap()
+    if len(dirs) > 4:
+        dm.num_dirs = 5
+    if expect:
+        with pytest.raises(scan.ScanError) as ei:
+            scan.selective_scan_workspace_size(sh, dm)
+        assert ei.value.status == expect
+    else:
+        assert scan.selective_scan_workspace_size(sh, dm) >= 0
+
+
+def test_null_alignment_and_workspace_errors():
+    sh = _shape()
+    args = [FAKE] * 5
+    # missing required pointers
+    for i in range(5):
+        a = list(args)
+        a[i] = 0
+        u, delta, A, B, C = a
+        st = scan.selective_scan_fwd_raw(sh, u, delta, A, B, C, 0, 0, 0, 1, None, FAKE, 0, 0, 0, 0)
+        assert st == 1
+    st = scan.selective_scan_fwd_raw(sh, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, 0, 1, None, 0, 0, 0, 0, 0)
+    assert st == 1
+    # misaligned io pointer / float pointer
+    st = scan.selective_scan_fwd_raw(sh, FAKE + 8, FAKE, FAKE, FAKE, FAKE, 0, 0, 0, 1, None, FAKE,
+                                     0, 0, 0, 0)
+    assert st == 4
+    st = scan.selective_scan_fwd_raw(sh, FAKE, FAKE, FAKE + 2, FAKE, FAKE, 0, 0, 0, 1, None, FAKE,
+                                     0, 0, 0, 0)
+    assert st == 4
+    # two directions need a workspace
+    dm = scan.make_dirmap((0, 1))
+    need = scan.selective_scan_workspace_size(sh, dm)
+    assert need > 0
+    st = scan.selective_scan_fwd_raw(sh, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, 0, 1, dm, FAKE, 0,
+                                     0, 0, 0)
+    assert st == 8
+    st = scan.selective_scan_fwd_raw(sh, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, 0, 1, dm, FAKE, 0,
+                                     FAKE, need - 1, 0)
+    assert st == 8
+    # unknown option bits / reserved fields
+    o = scan.make_opts(flags=2)
+    with pytest.raises(scan.ScanError):
+        scan.selective_scan_workspace_size(sh, None, o)
+    o = scan.make_opts(segments=-1)
+    with pytest.raises(scan.ScanError):
+        scan.selective_scan_workspace_size(sh, None, o)
+
+
+def test_workspace_sizes():
+    # one direction, one segment: no scratch
+    assert scan.selective_scan_workspace_size(_shape(), None, scan.make_opts(segments=1)) == 0
+    # segments: carries of K*b*S*D*(N+1) floats
+    n = scan.selective_scan_workspace_size(_shape(seqlen=4096), None, scan.make_opts(segments=4))
+    assert n >= 2 * 4 * 32 * 17 * 4
+    # directions: per-direction fp32 outputs
+    n = scan.selective_scan_workspace_size(_shape(), scan.make_dirmap((0, 1)))
+    assert n >= 2 * 2 * 64 * 32 * 4
+
+
+def test_empty_problem_needs_no_pointers():
+    for kw in (dict(batch=0), dict(seqlen=0), dict(dim=0)):
+        sh = _shape(**kw)
+        st = scan.selective_scan_fwd_raw(sh, 0, 0, FAKE if kw.get("dim", 1) else 0, 0, 0, 0, 0, 0,
+                                         1, None, 0, 0, 0, 0, 0)
+        assert st == 0, kw
+
+
+@pytest.mark.parametrize("H,W", [(56, 56), (5, 7), (1, 13), (13, 1), (3, 200)])
+def test_index_map_bit_exact_against_oracle(H, W):
+    L = H * W
+    dm = scan.make_dirmap((0, 1, 2, 3), H, W)
+    for k, d in enumerate((0, 1, 2, 3)):
+        got = [scan.ss_direction_position(dm, k, L, t) for t in range(L)]
+        ref = [oracle.position(d, L, t, H, W) for t in range(L)]
+        assert got == ref
+        assert sorted(got) == list(range(L))
+    assert scan.ss_direction_position(dm, 4, L, 0) == -1
+    assert scan.ss_direction_position(dm, 0, L, L) == -1
+    assert scan.ss_direction_position(None, 0, L, 3) == 3
+
+
+def test_index_map_large_L():
+    L = 131072
+    for t in (0, 1, 65535, L - 1):
+        assert scan.ss_direction_position(None, 0, L, t) == t
+        dm = scan.make_dirmap((1,))
+        assert scan.ss_direction_position(dm, 0, L, t) == L - 1 - t

@@ -1,0 +1,176 @@
+"""Parity of the CUDA selective scan with the fp64 oracle (needs a B200).
+
+Small cases are compared element by element: they span several channel tiles and time tiles,
+ragged channel and time tails, every state count up to 16, one to four directions, split
+sequences, the generic-A path, softplus off with Delta = 0 steps, and missing optional inputs.
+The five full-size workloads run in the launch configuration the benchmark times and are
+compared on sampled channels (every step of every sampled channel, which the oracle computes
+independently per channel).  Bars: max relative error (floor 1e-2 * rms) <= 1e-4 for fp32
+inputs, <= 2e-2 for bf16 inputs with fp32 state.
+"""
+
+import numpy as np
+import pytest
+
+from selective_state_space_13_b200 import workloads as wl
+from tests.scan_util import (TOL_BF16, TOL_F32, out_to_f64, rel_err, run_gpu, run_oracle,
+                             to_device, tol_for)
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(inp, device, tol=None, **kw):
+    w = inp["workload"]
+    opts = {k: kw.pop(k) for k in ("segments", "flags") if k in kw}
+    out, last = run_gpu(inp, device=device, **opts, **kw)
+    ref_out, ref_last = run_oracle(inp, **kw)
+    tol = tol_for(w) if tol is None else tol
+    e_out = rel_err(out_to_f64(out), ref_out)
+    e_last = rel_err(out_to_f64(last), ref_last)
+    assert e_out <= tol and e_last <= tol, (w.name, e_out, e_last)
+    return e_out, e_last
+
+
+def test_tiny_workload(cuda_device):
+    _check(wl.make_inputs("tiny"), cuda_device)
+
+
+@pytest.mark.parametrize("segments", [0, 1, 3])
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F32])
+def test_single_direction_ragged(cuda_device, dtype, segments):
+    w = wl.variant("m130", name="small", batch=2, seqlen=300, dim=136, dtype=dtype, seed=71)
+    _check(wl.make_inputs(w), cuda_device, segments=segments)
+
+
+@pytest.mark.parametrize("N", [1, 3, 4, 5, 8, 11, 16])
+def test_state_sizes(cuda_device, N):
+    w = wl.variant("m130", name="nstate", batch=2, seqlen=97, dim=72, dstate=N, seed=100 + N)
+    _check(wl.make_inputs(w), cuda_device)
+
+
+@pytest.mark.parametrize("flags", [0, 1])
+def test_generic_A(cuda_device, flags):
+    w = wl.variant("m130", name="genA", batch=2, seqlen=130, dim=64, dtype=wl.F32, seed=81)
+    inp = wl.make_inputs(w)
+    if flags == 0:
+        rng = np.random.default_rng(5)
+        inp["A"] = (-rng.uniform(0.05, 3.0, size=inp["A"].shape)).astype(np.float32)
+    _check(inp, cuda_device, flags=flags)
+
+
+def test_mixed_chain_and_generic_channels(cuda_device):
+    # some channels satisfy A[d,n] = (n+1) A[d,0], others do not, inside one warp
+    w = wl.variant("m130", name="mixA", batch=1, seqlen=77, dim=64, dtype=wl.F32, seed=82)
+    inp = wl.make_inputs(w)
+    inp["A"][::3] *= np.float32(0.37)  # still a chain
+    inp["A"][1::5, 2] = np.float32(-0.123)  # breaks the chain for these channels
+    _check(inp, cuda_device)
+
+
+@pytest.mark.parametrize("L", [1, 2, 31, 32, 33, 65])
+def test_short_sequences(cuda_device, L):
+    w = wl.variant("m130", name="short", batch=3, seqlen=L, dim=40, seed=90 + L)
+    _check(wl.make_inputs(w), cuda_device)
+
+
+def test_vim_like_bidirectional(cuda_device):
+    w = wl.variant("vim", name="vim_small", batch=3, dim=64, seed=91)
+    _check(wl.make_inputs(w), cuda_device)
+
+
+@pytest.mark.parametrize("segments", [0, 2])
+def test_ss2d_like_cross_scan(cuda_device, segments):
+    w = wl.variant("ss2d", name="ss2d_small", batch=2, seqlen=120, H=12, W=10, dim=32, seed=92)
+    _check(wl.make_inputs(w), cuda_device, segments=segments)
+
+
+def test_directions_fp32_gate(cuda_device):
+    w = wl.Workload("dirs32", 2, 48, 16, 4, wl.F32, dirs=(wl.DIR_COLUMN_REVERSE, wl.DIR_REVERSE,
+                                                          wl.DIR_COLUMN), H=6, W=8, seed=93,
+                    dskip="normal")
+    _check(wl.make_inputs(w), cuda_device)
+
+
+def test_optional_inputs_absent(cuda_device):
+    w = wl.variant("m130", name="opt", batch=2, seqlen=70, dim=48, seed=94)
+    inp = wl.make_inputs(w)
+    _check(inp, cuda_device, use_z=False, use_D=False, use_bias=False)
+
+
+def test_softplus_off_zero_delta_steps(cuda_device):
+    w = wl.variant("m130", name="dz", batch=2, seqlen=90, dim=32, dtype=wl.F32, seed=95)
+    inp = wl.make_inputs(w)
+    rng = np.random.default_rng(6)
+    # Delta = delta + bias; positive steps, with some steps exactly zero
+    inp["delta"] = rng.uniform(0.01, 0.4, size=inp["delta"].shape).astype(np.float32)
+    inp["delta"] -= inp["delta_bias"][None, None, None, :]
+    zero = [0, 1, 17, 40, 41, 42, 89]
+    inp["delta"][:, :, zero, :] = -inp["delta_bias"][None, None, :]
+    _check(inp, cuda_device, softplus=False)
+
+
+def test_empty_problems(cuda_device):
+    import torch
+    from selective_state_space_13_b200 import scan
+    for batch, L in ((0, 16), (2, 0)):
+        u = torch.empty((batch, L, 16), device=cuda_device)
+        d = torch.empty((1, batch, L, 16), device=cuda_device)
+        bc = torch.empty((1, batch, L, 4), device=cuda_device)
+        A = -torch.ones((16, 4), device=cuda_device)
+        out, last = scan.selective_scan_fwd(u, d, A, bc, bc, return_last_state=True)
+        torch.cuda.synchronize()
+        assert out.shape == u.shape
+        if L == 0 and batch:
+            assert torch.all(last == 0)
+
+
+def test_repeat_calls_identical(cuda_device):
+    # the scan is deterministic: two calls give bit-identical results
+    w = wl.variant("m130", name="rep", batch=2, seqlen=200, dim=64, seed=96)
+    inp = wl.make_inputs(w)
+    t = to_device(inp, cuda_device)
+    o1, l1 = run_gpu(inp, dev_inputs=t, segments=2)
+    o2, l2 = run_gpu(inp, dev_inputs=t, segments=2)
+    assert bool((o1 == o2).all()) and bool((l1 == l2).all())
+
+
+def test_device_status_clean(cuda_device):
+    from selective_state_space_13_b200 import scan
+    assert scan.selective_scan_device_status(clear=True) == scan.SS_OK
+
+
+# ----------------------------------------------------------------------------- full size
+
+FULL_SAMPLES = {
+    # workload: (batch rows sampled, channels sampled)
+    "tiny": (None, None),
+    "m130": (None, 24),
+    "long": (None, 64),
+    "vim": (8, 32),
+    "ss2d": (4, 16),
+}
+
+
+@pytest.mark.parametrize("name", ["tiny", "m130", "long", "vim", "ss2d"])
+def test_full_size_workloads_sampled(cuda_device, name):
+    import torch
+    w = wl.WORKLOADS[name]
+    inp = wl.make_inputs(w)
+    t = to_device(inp, cuda_device)
+    out, last = run_gpu(inp, dev_inputs=t)            # default launch = the benchmark's
+    torch.cuda.synchronize()
+    nb, nc = FULL_SAMPLES[name]
+    rng = np.random.default_rng(7)
+    bsel = None if nb is None else np.sort(rng.choice(w.batch, size=nb, replace=False))
+    csel = None if nc is None else np.sort(rng.choice(w.dim, size=nc, replace=False))
+    ref_out, ref_last = run_oracle(inp, channels=csel, batches=bsel)
+    bi = torch.arange(w.batch) if bsel is None else torch.from_numpy(bsel)
+    ci = torch.arange(w.dim) if csel is None else torch.from_numpy(csel)
+    got = out.index_select(0, bi.to(out.device)).index_select(2, ci.to(out.device))
+    got_last = last.index_select(1, bi.to(out.device)).index_select(2, ci.to(out.device))
+    e_out = rel_err(out_to_f64(got), ref_out)
+    e_last = rel_err(out_to_f64(got_last), ref_last)
+    tol = TOL_F32 if w.dtype == wl.F32 else TOL_BF16
+    del t, out, last, got, got_last
+    torch.cuda.empty_cache()
+    assert e_out <= tol and e_last <= tol, (name, e_out, e_last)
