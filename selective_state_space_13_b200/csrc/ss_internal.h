@@ -4,6 +4,7 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "selective_scan.h"
@@ -11,11 +12,17 @@
 namespace ss {
 
 // Steps per pipeline stage and number of stages of the shared-memory ring.
-constexpr int kTile = 32;
+constexpr int kTile = 16;
 constexpr int kStages = 4;
+// Rows whose per-step scalars the fast path computes together.
+constexpr int kGroup = 8;
 
 // Everything a scan launch needs.  Device pointers are the caller's; nothing here is owned.
+// The tensor maps are filled in by launch_scan.
 struct ScanParams {
+    CUtensorMap tm_u, tm_z;    // u, z as [batch*L rows, D]: boxes of kTile rows x DC channels
+    CUtensorMap tm_dl;         // delta as [K*batch*L rows, D], same boxes
+    CUtensorMap tm_u3, tm_z3;  // u, z as [batch*H, W, D]: boxes of 8 image rows of one column
     const void* u;          // [batch, L, D] io, spatial order
     const void* delta;      // [K, batch, L, D] io, scan order
     const float* A;         // [D, N]
@@ -36,6 +43,7 @@ struct ScanParams {
     int32_t H, W;
     int32_t softplus;
     int32_t force_generic;  // 1: never take the A[d,n] = (n+1) A[d,0] shortcut
+    int32_t col3d;          // 1: column orders load through tm_u3 / tm_z3 (H % 8 == 0)
 };
 
 struct MergeParams {

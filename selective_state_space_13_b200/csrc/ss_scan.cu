@@ -33,10 +33,13 @@
 // Every wait on an mbarrier is bounded in time.  A wait that gives up sets the library's device
 // error word (read by selective_scan_device_status), waits a bounded time for the copies this
 // CTA still has in flight, and the whole CTA returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "ss_internal.h"
 
@@ -128,6 +131,28 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
+// Tiled tensor copies global -> shared through a tensor map (a __grid_constant__ parameter);
+// coordinates are in elements, innermost first.
+__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, int32_t c0, int32_t c1,
+                                       uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_3d(void* dst, const CUtensorMap* map, int32_t c0, int32_t c1,
+                                       int32_t c2, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ float ex2(float x)
 {
     float y;
@@ -147,6 +172,40 @@ __device__ __forceinline__ float rcp(float x)
     float y;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// log(1 + e) for e in [0, 1], relative error ~1e-7: 2*atanh(s) with s = e / (2 + e) <= 1/3,
+// odd series up to s^15 (truncation < 2e-9 relative).
+__device__ __forceinline__ float log1p_unit(float e)
+{
+    const float s = e * rcp(2.f + e);
+    const float s2 = s * s;
+    float p = 2.f / 15.f;
+    p = fmaf(p, s2, 2.f / 13.f);
+    p = fmaf(p, s2, 2.f / 11.f);
+    p = fmaf(p, s2, 2.f / 9.f);
+    p = fmaf(p, s2, 2.f / 7.f);
+    p = fmaf(p, s2, 2.f / 5.f);
+    p = fmaf(p, s2, 2.f / 3.f);
+    p = fmaf(p, s2, 2.f);
+    return s * p;
+}
+
+// exp(x) - 1 with relative accuracy ~1e-7 near 0 (Taylor to x^8 for |x| <= 0.35, truncation
+// < 3e-10 relative), exp through ex2 elsewhere.
+__device__ __forceinline__ float expm1_acc(float x)
+{
+    float p = 1.f / 40320.f;
+    p = fmaf(p, x, 1.f / 5040.f);
+    p = fmaf(p, x, 1.f / 720.f);
+    p = fmaf(p, x, 1.f / 120.f);
+    p = fmaf(p, x, 1.f / 24.f);
+    p = fmaf(p, x, 1.f / 6.f);
+    p = fmaf(p, x, 0.5f);
+    p = fmaf(p, x, 1.f);
+    const float small = x * p;
+    const float big = ex2(x * 1.4426950408889634f) - 1.f;
+    return fabsf(x) <= 0.35f ? small : big;
 }
 
 // ---------------------------------------------------------------------------- element types
@@ -184,6 +243,8 @@ __host__ __device__ __forceinline__ int64_t position(int32_t dir, int64_t L, int
 
 // ---------------------------------------------------------------------------- shared layout
 
+// One pipeline stage holds kTile rows of u, delta and z for the CTA's channels (as copied),
+// the raw B and C tiles, their fp32 copies, and the output row offsets of the tile.
 template <typename io_t, int NS, int WARPS, bool GATE, bool PHASE1>
 struct Layout {
     static constexpr int DC = 32 * WARPS;                           // channels per CTA
@@ -197,30 +258,39 @@ struct Layout {
     static constexpr int OFF_Z = OFF_DL + ROWS;
     static constexpr int OFF_BR = OFF_Z + (HAS_Z ? ROWS : 0);
     static constexpr int OFF_CR = OFF_BR + BCRAW;
-    static constexpr int OFF_POS = OFF_CR + (HAS_C ? BCRAW : 0);
-    static constexpr int STAGE = ((OFF_POS + kTile * 4 + 127) / 128) * 128;
-    static constexpr int OFF_BC = kStages * STAGE;                   // fp32 B (and C), 2 buffers
-    static constexpr int BC_ONE = kTile * NS * 4;
-    static constexpr int BC_BUF = BC_ONE * (HAS_C ? 2 : 1);
-    static constexpr int OFF_BAR = OFF_BC + 2 * BC_BUF;
-    static constexpr int OFF_FLAG = OFF_BAR + kStages * 8;
+    static constexpr int OFF_BF = OFF_CR + (HAS_C ? BCRAW : 0);      // fp32 B, then fp32 C
+    static constexpr int BF_ONE = kTile * NS * 4;
+    static constexpr int OFF_OUT = OFF_BF + BF_ONE * (HAS_C ? 2 : 1);  // int64 row offsets
+    static constexpr int STAGE = ((OFF_OUT + kTile * 8 + 127) / 128) * 128;
+    static constexpr int OFF_BAR = kStages * STAGE;                  // full, ready, empty
+    static constexpr int OFF_FLAG = OFF_BAR + 3 * kStages * 8;
     static constexpr int BYTES = OFF_FLAG + 16;
-    static_assert(ROW % 16 == 0 && BCRAW % 16 == 0 && OFF_POS % 16 == 0, "TMA destinations");
-    static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");
+    static_assert(ROW % 16 == 0 && BCRAW % 16 == 0 && OFF_BF % 16 == 0 && OFF_OUT % 8 == 0,
+                  "TMA destinations and vector accesses need 16-byte alignment");
 };
 
 // ---------------------------------------------------------------------------- the scan kernel
+//
+// Pipeline of one CTA (WARPS warps, every warp scans; warp 0 also produces):
+//   full[s]  completes when the bulk copies of the tile in stage s have landed (tx count);
+//   ready[s] completes when warp 0 has converted that tile's B and C to fp32;
+//   empty[s] completes when all WARPS warps are done with the tile in stage s.
+// Warp 0 refills the stage released two tiles earlier, so kStages-2 tiles are in flight
+// ahead of the one being scanned, and no warp other than warp 0 ever waits for another.
 
-template <typename io_t, int NS, int WARPS, bool GATE, bool PHASE1>
+template <typename io_t, int NS, int WARPS, bool GATE, bool PHASE1, bool YPART>
 __global__ void __launch_bounds__(32 * WARPS)
     scan_kernel(const __grid_constant__ ScanParams p)
 {
     using Lay = Layout<io_t, NS, WARPS, GATE, PHASE1>;
+    // fp32 inputs take the precise arithmetic, bf16 inputs the fast one
+    constexpr bool PRECISE = sizeof(io_t) == 4;
     constexpr int DC = Lay::DC;
-    constexpr int NT = 32 * WARPS;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
-    volatile int& s_abort = *reinterpret_cast<int*>(smem + Lay::OFF_FLAG);
+    uint64_t* ready = full + kStages;
+    uint64_t* empty = ready + kStages;
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Lay::OFF_FLAG);
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -236,7 +306,8 @@ __global__ void __launch_bounds__(32 * WARPS)
     blk /= nseg;
     const int64_t b = blk % p.batch;
     const int k = static_cast<int>(blk / p.batch);
-    const int dir = p.dirs[k];
+    // constant indices keep the parameter array out of local memory
+    const int dir = k == 0 ? p.dirs[0] : k == 1 ? p.dirs[1] : k == 2 ? p.dirs[2] : p.dirs[3];
 
     const int64_t d0 = tile * DC;
     const int dcv = static_cast<int>((p.D - d0) < DC ? (p.D - d0) : DC);  // valid channels
@@ -246,26 +317,28 @@ __global__ void __launch_bounds__(32 * WARPS)
     const int64_t t_end = (t_begin + p.seg_len < p.L) ? (t_begin + p.seg_len) : p.L;
     const int64_t ntile_t = (t_end - t_begin + kTile - 1) / kTile;
 
-    const int esz = static_cast<int>(sizeof(io_t));
-    const uint32_t row_bytes = static_cast<uint32_t>(dcv) * esz;
-
+    const uint32_t row_bytes = static_cast<uint32_t>(dcv) * static_cast<uint32_t>(sizeof(io_t));
     const io_t* gu = static_cast<const io_t*>(p.u);
     const io_t* gz = static_cast<const io_t*>(p.z);
-    const io_t* gdl = static_cast<const io_t*>(p.delta);
     const io_t* gB = static_cast<const io_t*>(p.B);
     const io_t* gC = static_cast<const io_t*>(p.C);
     const int64_t kb = static_cast<int64_t>(k) * p.batch + b;  // (direction, batch) row block
+    // output rows: out[b, p, :] for one direction, ypart[k, b, p, :] for several
+    const int64_t out_row0 = p.ypart ? kb * p.L : b * p.L;
 
     if (tid == 0) {
-        s_abort = 0;
-        for (int s = 0; s < kStages; ++s)
+        *s_abort = 0;
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&ready[s], 1);
+            mbar_init(&empty[s], WARPS);
+        }
         fence_mbar_init();
     }
     __syncthreads();
 
-    // B/C tiles are copied from a 16-byte aligned superset of their rows; this is the offset of
-    // the first wanted element inside the copied block.
+    // B/C tiles are copied from a 16-byte aligned superset of their rows; `skip` is the offset
+    // (in elements) of the first wanted element inside the copied block.
     auto bc_src = [&](const io_t* base, int64_t t0, int rows, uint32_t& bytes, int& skip) {
         const uintptr_t a0 = reinterpret_cast<uintptr_t>(base + (kb * p.L + t0) * p.N);
         const uintptr_t a1 = reinterpret_cast<uintptr_t>(base + (kb * p.L + t0 + rows) * p.N);
@@ -275,49 +348,117 @@ __global__ void __launch_bounds__(32 * WARPS)
         skip = static_cast<int>((a0 - lo) / sizeof(io_t));
         return reinterpret_cast<const void*>(lo);
     };
+    auto tile_rows = [&](int64_t it) {
+        const int64_t t0 = t_begin + it * kTile;
+        return static_cast<int>((t_end - t0) < kTile ? (t_end - t0) : kTile);
+    };
 
-    // Fill stage `st` with time tile `it` (warp 0 only; all 32 lanes issue copies).
-    auto issue = [&](int64_t it, int st) {
+    // How u and z rows reach shared memory: 0 = one box of kTile spatial rows (forward and
+    // reverse orders visit contiguous rows), 1 = boxes of 8 rows of one image column (column
+    // orders, H % 8 == 0), 2 = one bulk copy per row.  Step t0 + r of a tile reads u/z row
+    // (r ^ xmask) of the stage; delta rows are always in scan order.
+    const int umode = (dir == SS_DIR_FWD || dir == SS_DIR_REV) ? 0 : (p.col3d ? 1 : 2);
+    const int xmask =
+        dir == SS_DIR_REV ? (kTile - 1) : (dir == SS_DIR_COL_REV && umode == 1 ? 7 : 0);
+    constexpr uint32_t kBox2 = static_cast<uint32_t>(DC) * kTile * sizeof(io_t);
+    constexpr uint32_t kBox3 = static_cast<uint32_t>(DC) * 8 * sizeof(io_t);
+    constexpr uint32_t kUZ = Lay::HAS_Z ? 2u : 1u;
+
+    // Fill the stage of time tile `it` (warp 0).
+    auto issue = [&](int64_t it) {
+        const int st = static_cast<int>(it % kStages);
         unsigned char* sb = smem + st * Lay::STAGE;
         const int64_t t0 = t_begin + it * kTile;
-        const int rows = static_cast<int>((t_end - t0) < kTile ? (t_end - t0) : kTile);
+        const int rows = tile_rows(it);
         uint32_t bbytes, cbytes = 0;
         int bskip, cskip;
         const void* bsrc = bc_src(gB, t0, rows, bbytes, bskip);
         const void* csrc = Lay::HAS_C ? bc_src(gC, t0, rows, cbytes, cskip) : nullptr;
         if (lane == 0) {
-            const uint32_t tx = static_cast<uint32_t>(rows) * row_bytes * (Lay::HAS_Z ? 3u : 2u) +
-                                bbytes + cbytes;
+            uint32_t tx = kBox2 + bbytes + cbytes;  // delta box, B, C
+            if (umode == 0)
+                tx += kUZ * kBox2;
+            else if (umode == 1)
+                tx += kUZ * kBox3 * static_cast<uint32_t>(rows / 8);
+            else
+                tx += kUZ * static_cast<uint32_t>(rows) * row_bytes;
             mbar_expect_tx(&full[st], tx);
-        }
-        __syncwarp();
-        int32_t* pos = reinterpret_cast<int32_t*>(sb + Lay::OFF_POS);
-        for (int r = lane; r < rows; r += 32) {
-            const int64_t t = t0 + r;
-            const int64_t pp = position(dir, p.L, p.H, p.W, t);
-            pos[r] = static_cast<int32_t>(pp);
-            bulk_g2s(sb + Lay::OFF_U + r * Lay::ROW, gu + (b * p.L + pp) * p.D + d0, row_bytes,
-                     &full[st]);
-            bulk_g2s(sb + Lay::OFF_DL + r * Lay::ROW, gdl + (kb * p.L + t) * p.D + d0, row_bytes,
-                     &full[st]);
-            if (Lay::HAS_Z)
-                bulk_g2s(sb + Lay::OFF_Z + r * Lay::ROW, gz + (b * p.L + pp) * p.D + d0, row_bytes,
-                         &full[st]);
-        }
-        if (lane == 0) {
+            tma_2d(sb + Lay::OFF_DL, &p.tm_dl, static_cast<int32_t>(d0),
+                   static_cast<int32_t>(kb * p.L + t0), &full[st]);
+            if (umode == 0) {
+                // reverse order: the box ends at the row of step t0
+                const int64_t prow = b * p.L + (dir == SS_DIR_FWD ? t0 : p.L - t0 - kTile);
+                tma_2d(sb + Lay::OFF_U, &p.tm_u, static_cast<int32_t>(d0),
+                       static_cast<int32_t>(prow), &full[st]);
+                if (Lay::HAS_Z)
+                    tma_2d(sb + Lay::OFF_Z, &p.tm_z, static_cast<int32_t>(d0),
+                           static_cast<int32_t>(prow), &full[st]);
+            } else if (umode == 1) {
+                for (int sub = 0; sub < rows / 8; ++sub) {
+                    const int64_t tt = t0 + 8 * sub;
+                    // column-major index of the lowest image row of the box
+                    const int64_t c = dir == SS_DIR_COL ? tt : (p.L - 8 - tt);
+                    const int64_t j = c / p.H, i = c - (c / p.H) * p.H;
+                    tma_3d(sb + Lay::OFF_U + 8 * sub * Lay::ROW, &p.tm_u3,
+                           static_cast<int32_t>(d0), static_cast<int32_t>(j),
+                           static_cast<int32_t>(b * p.H + i), &full[st]);
+                    if (Lay::HAS_Z)
+                        tma_3d(sb + Lay::OFF_Z + 8 * sub * Lay::ROW, &p.tm_z3,
+                               static_cast<int32_t>(d0), static_cast<int32_t>(j),
+                               static_cast<int32_t>(b * p.H + i), &full[st]);
+                }
+            }
             bulk_g2s(sb + Lay::OFF_BR, bsrc, bbytes, &full[st]);
             if (Lay::HAS_C)
                 bulk_g2s(sb + Lay::OFF_CR, csrc, cbytes, &full[st]);
+        }
+        __syncwarp();
+        int64_t* orow = reinterpret_cast<int64_t*>(sb + Lay::OFF_OUT);
+        for (int r = lane; r < rows; r += 32) {
+            const int64_t pp = position(dir, p.L, p.H, p.W, t0 + r);
+            orow[r] = (out_row0 + pp) * p.D + d0;
+            if (umode == 2) {
+                bulk_g2s(sb + Lay::OFF_U + r * Lay::ROW, gu + (b * p.L + pp) * p.D + d0,
+                         row_bytes, &full[st]);
+                if (Lay::HAS_Z)
+                    bulk_g2s(sb + Lay::OFF_Z + r * Lay::ROW, gz + (b * p.L + pp) * p.D + d0,
+                             row_bytes, &full[st]);
+            }
         }
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&full[st]);
     };
 
+    // Convert tile `it`'s B (and C) to fp32 (warp 0).  On the fast path B carries the ln 2 of
+    // w = Delta*u / ln 2.
+    auto convert = [&](int64_t it) {
+        const int st = static_cast<int>(it % kStages);
+        unsigned char* sb = smem + st * Lay::STAGE;
+        const int64_t t0 = t_begin + it * kTile;
+        const int rows = tile_rows(it);
+        uint32_t bytes;
+        int bskip = 0, cskip = 0;
+        bc_src(gB, t0, rows, bytes, bskip);
+        if (Lay::HAS_C)
+            bc_src(gC, t0, rows, bytes, cskip);
+        const io_t* br = reinterpret_cast<const io_t*>(sb + Lay::OFF_BR) + bskip;
+        const io_t* cr = reinterpret_cast<const io_t*>(sb + Lay::OFF_CR) + cskip;
+        float* bf = reinterpret_cast<float*>(sb + Lay::OFF_BF);
+        const float bscale = PRECISE ? 1.f : kLn2;
+        for (int idx = lane; idx < kTile * NS; idx += 32) {
+            const int r = idx / NS, n = idx - (idx / NS) * NS;
+            const bool ok = r < rows && n < p.N;
+            bf[idx] = ok ? Io<io_t>::ld(br + r * p.N + n) * bscale : 0.f;
+            if (Lay::HAS_C)
+                bf[kTile * NS + idx] = ok ? Io<io_t>::ld(cr + r * p.N + n) : 0.f;
+        }
+    };
+
     // ---- per-channel constants
     float a_l[NS];       // A[d, n] (natural units; multiplies Delta*log2(e))
     bool chain = true;   // A[d, n] == (n+1) * A[d, 0] for all n
-    float dskip = 0.f, bias2 = 0.f;
+    float dskip = 0.f, bias2 = 0.f, bias_raw = 0.f;
     if (active) {
 #pragma unroll
         for (int n = 0; n < NS; ++n) {
@@ -326,20 +467,23 @@ __global__ void __launch_bounds__(32 * WARPS)
                 chain = false;
         }
         dskip = p.Dskip ? p.Dskip[d] : 0.f;
-        bias2 = (p.bias ? p.bias[d] : 0.f) * kLog2e;
+        bias_raw = p.bias ? p.bias[d] : 0.f;
+        bias2 = bias_raw * kLog2e;
     } else {
 #pragma unroll
         for (int n = 0; n < NS; ++n)
             a_l[n] = 0.f;
     }
     const bool use_chain = __all_sync(0xffffffffu, chain) && !p.force_generic;
+    const bool softplus = p.softplus != 0;
 
-    // ---- state: normalised k = h / w_prev
-    float kst[NS];
+    // ---- state, as pairs (n, n+1): the fast path keeps k = h / w_prev, the precise path h
+    float2 kst2[NS / 2];
+    float* kst = reinterpret_cast<float*>(kst2);
     float wprev = 1.f;
 #pragma unroll
-    for (int n = 0; n < NS; ++n)
-        kst[n] = 0.f;
+    for (int j = 0; j < NS / 2; ++j)
+        kst2[j] = make_float2(0.f, 0.f);
     if (!PHASE1 && seg > 0 && active) {
         // fold the carries of segments 0..seg-1: h <- exp(A * sumDelta_s) * h + h_s
         for (int s = 0; s < seg; ++s) {
@@ -354,84 +498,75 @@ __global__ void __launch_bounds__(32 * WARPS)
     }
     float dsum = 0.f;  // sum of Delta*log2(e) over this segment (aggregate launch)
 
-    // ---- prologue: fill kStages-1 stages
+    // ---- prologue: warp 0 fills the first kStages-2 stages
     int64_t issued = 0;
-    if (warp == 0) {
-        for (; issued < kStages - 1 && issued < ntile_t; ++issued)
-            issue(issued, static_cast<int>(issued % kStages));
-    }
+    if (warp == 0)
+        for (; issued < kStages - 2 && issued < ntile_t; ++issued)
+            issue(issued);
 
-    float* bcbuf = reinterpret_cast<float*>(smem + Lay::OFF_BC);
-    int64_t failed_at = -1;
+    bool failed = false;
     for (int64_t it = 0; it < ntile_t; ++it) {
         const int st = static_cast<int>(it % kStages);
-        const uint32_t parity = static_cast<uint32_t>((it / kStages) & 1);
+        const uint32_t ph = static_cast<uint32_t>((it / kStages) & 1);
         unsigned char* sb = smem + st * Lay::STAGE;
-        const int64_t t0 = t_begin + it * kTile;
-        const int rows = static_cast<int>((t_end - t0) < kTile ? (t_end - t0) : kTile);
-
-        if (!mbar_wait_bounded(&full[st], parity, kWaitLimitNs)) {
-            atomicOr(&g_ss_status, kStatusTimeout);
-            s_abort = 1;
-        }
-        // convert this tile's B (and C) to fp32; B carries the ln 2 of w = Delta*u
-        float* bf = bcbuf + (it & 1) * (Lay::BC_BUF / 4);
-        {
-            uint32_t bbytes, cbytes = 0;
-            int bskip = 0, cskip = 0;
-            bc_src(gB, t0, rows, bbytes, bskip);
-            if (Lay::HAS_C)
-                bc_src(gC, t0, rows, cbytes, cskip);
-            const io_t* br = reinterpret_cast<const io_t*>(sb + Lay::OFF_BR) + bskip;
-            const io_t* cr = reinterpret_cast<const io_t*>(sb + Lay::OFF_CR) + cskip;
-            for (int idx = tid; idx < kTile * NS; idx += NT) {
-                const int r = idx / NS, n = idx - (idx / NS) * NS;
-                const bool ok = r < rows && n < p.N;
-                bf[idx] = ok ? Io<io_t>::ld(br + r * p.N + n) * kLn2 : 0.f;
-                if (Lay::HAS_C)
-                    bf[kTile * NS + idx] = ok ? Io<io_t>::ld(cr + r * p.N + n) : 0.f;
-            }
-        }
-        __syncthreads();  // tile `it` converted; every thread is done with tile it-1
-        if (s_abort) {
-            failed_at = it;
+        const int rows = tile_rows(it);
+        if (*s_abort) {
+            failed = true;
             break;
         }
-        if (warp == 0 && issued < ntile_t) {
-            issue(issued, static_cast<int>(issued % kStages));
-            ++issued;
+        if (warp == 0) {
+            if (!mbar_wait_bounded(&full[st], ph, kWaitLimitNs)) {
+                failed = true;
+            } else {
+                convert(it);
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&ready[st]);
+                // refill the stage released two tiles ago
+                const int64_t nx = it + kStages - 2;
+                if (nx < ntile_t) {
+                    if (nx >= kStages &&
+                        !mbar_wait_bounded(&empty[nx % kStages],
+                                           static_cast<uint32_t>(((nx / kStages) - 1) & 1),
+                                           kWaitLimitNs))
+                        failed = true;
+                    else
+                        issue(nx);
+                    issued = nx + 1;
+                }
+            }
+        } else {
+            if (!mbar_wait_bounded(&ready[st], ph, kWaitLimitNs) ||
+                !mbar_wait_bounded(&full[st], ph, kWaitLimitNs))
+                failed = true;
+        }
+        if (failed) {
+            atomicOr(&g_ss_status, kStatusTimeout);
+            *s_abort = 1;
+            break;
         }
 
         if (active) {
             const io_t* su = reinterpret_cast<const io_t*>(sb + Lay::OFF_U);
             const io_t* sdl = reinterpret_cast<const io_t*>(sb + Lay::OFF_DL);
             const io_t* sz = reinterpret_cast<const io_t*>(sb + Lay::OFF_Z);
-            const int32_t* pos = reinterpret_cast<const int32_t*>(sb + Lay::OFF_POS);
+            const int64_t* orow = reinterpret_cast<const int64_t*>(sb + Lay::OFF_OUT);
+            const float* bf = reinterpret_cast<const float*>(sb + Lay::OFF_BF);
             const float4* B4 = reinterpret_cast<const float4*>(bf);
             const float4* C4 = reinterpret_cast<const float4*>(bf + kTile * NS);
-            for (int r = 0; r < rows; ++r) {
-                const float uv = Io<io_t>::ld(su + r * DC + tid);
-                const float dr = Io<io_t>::ld(sdl + r * DC + tid);
-                // x = (delta + bias) * log2(e); Delta*log2(e) = softplus in base 2 of x
-                const float x = fmaf(dr, kLog2e, bias2);
-                float sp2 = x;
-                if (p.softplus) {
-                    const float e = ex2(-fabsf(x));              // 2^-|x| in (0, 1]
-                    const float l_big = lg2(1.f + e);
-                    // log2(1+e) for small e: e*log2(e)*(1 - e/2), relative error < e^2/3
-                    const float l_small = e * fmaf(e, -0.5f * kLog2e, kLog2e);
-                    sp2 = fmaxf(x, 0.f) + (e < 0.00390625f ? l_small : l_big);
-                }
-                float w = sp2 * uv;                               // = Delta*u / ln 2
-                w = fabsf(w) < kTinyW ? kTinyW : w;
-                const float rr = wprev * rcp(w);
-                wprev = w;
-                if (PHASE1)
-                    dsum += sp2;
-                float yp = 0.f;
-                if (use_chain) {
-                    const float q = ex2(sp2 * a_l[0]);
-                    float c = rr;
+            if (PRECISE) {
+                // h = (1 + expm1(Delta*A)) h + Delta*u*B without rounding Abar to fp32, so the
+                // per-step error does not grow with the memory length 1/|Delta*A|
+                for (int r = 0; r < rows; ++r) {
+                    const float uv = Io<io_t>::ld(su + (r ^ xmask) * DC + tid);
+                    const float dr = Io<io_t>::ld(sdl + r * DC + tid);
+                    const float x = dr + bias_raw;
+                    const float spv = fmaxf(x, 0.f) + log1p_unit(ex2(-fabsf(x) * kLog2e));
+                    const float dt = softplus ? spv : x;
+                    const float w = dt * uv;
+                    if (PHASE1)
+                        dsum += dt * kLog2e;
+                    float yp = 0.f;
 #pragma unroll
                     for (int n4 = 0; n4 < NS / 4; ++n4) {
                         const float4 bq = B4[r * (NS / 4) + n4];
@@ -443,57 +578,148 @@ __global__ void __launch_bounds__(32 * WARPS)
                         }
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            c *= q;
-                            kst[n4 * 4 + j] = fmaf(c, kst[n4 * 4 + j], bv[j]);
+                            const int n = n4 * 4 + j;
+                            const float em1 = expm1_acc(dt * a_l[n]);
+                            kst[n] = fmaf(em1, kst[n], fmaf(w, bv[j], kst[n]));
                             if (!PHASE1)
-                                yp = fmaf(cv[j], kst[n4 * 4 + j], yp);
+                                yp = fmaf(cv[j], kst[n], yp);
                         }
                     }
-                } else {
-#pragma unroll
-                    for (int n4 = 0; n4 < NS / 4; ++n4) {
-                        const float4 bq = B4[r * (NS / 4) + n4];
-                        const float bv[4] = {bq.x, bq.y, bq.z, bq.w};
-                        float cv[4] = {0.f, 0.f, 0.f, 0.f};
-                        if (!PHASE1) {
-                            const float4 cq = C4[r * (NS / 4) + n4];
-                            cv[0] = cq.x; cv[1] = cq.y; cv[2] = cq.z; cv[3] = cq.w;
-                        }
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float c = rr * ex2(sp2 * a_l[n4 * 4 + j]);
-                            kst[n4 * 4 + j] = fmaf(c, kst[n4 * 4 + j], bv[j]);
-                            if (!PHASE1)
-                                yp = fmaf(cv[j], kst[n4 * 4 + j], yp);
+                    if (!PHASE1) {
+                        float y = fmaf(dskip, uv, yp);
+                        if (YPART) {
+                            p.ypart[orow[r] + tid] = y;
+                        } else {
+                            if (GATE) {
+                                const float zv = Io<io_t>::ld(sz + (r ^ xmask) * DC + tid);
+                                y *= zv / (1.f + ex2(-zv * kLog2e));
+                            }
+                            static_cast<io_t*>(p.out)[orow[r] + tid] = Io<io_t>::st(y);
                         }
                     }
                 }
-                if (!PHASE1) {
-                    float y = fmaf(dskip, uv, w * yp);
-                    const int64_t pp = pos[r];
-                    if (p.ypart) {
-                        p.ypart[(kb * p.L + pp) * p.D + d] = y;
-                    } else {
+            } else {
+                // fast path, kGroup rows at a time: first the per-step scalars of all kGroup
+                // rows, then their state updates; no branch inside a group, so the compiler can
+                // overlap consecutive rows.  A row past the tile's end leaves the state as it
+                // is: q = 1, w = the previous w (so w_prev/w = 1), and B = 0 there.
+                auto group = [&](auto chain_tag, int r0) {
+                    constexpr bool CHAIN = decltype(chain_tag)::value;
+                    float s_q[kGroup], s_w[kGroup], s_rr[kGroup], s_sp[kGroup], s_du[kGroup],
+                        s_g[kGroup];
+#pragma unroll
+                    for (int g = 0; g < kGroup; ++g) {
+                        const bool valid = r0 + g < rows;
+                        const int r = valid ? (r0 + g) : (rows - 1);
+                        const float uv = Io<io_t>::ld(su + (r ^ xmask) * DC + tid);
+                        const float dr = Io<io_t>::ld(sdl + r * DC + tid);
+                        // x = (delta + bias) * log2(e); Delta*log2(e) = softplus in base 2 of x
+                        const float x = fmaf(dr, kLog2e, bias2);
+                        const float e = ex2(-fabsf(x));              // 2^-|x| in (0, 1]
+                        const float l_big = lg2(1.f + e);
+                        // log2(1+e) for small e: e*log2(e)*(1 - e/2), rel. error < e^2/3
+                        const float l_small = e * fmaf(e, -0.5f * kLog2e, kLog2e);
+                        const float spv = fmaxf(x, 0.f) + (e < 0.00390625f ? l_small : l_big);
+                        const float sp2 = valid ? (softplus ? spv : x) : 0.f;
+                        float w = sp2 * uv;                           // = Delta*u / ln 2
+                        w = fabsf(w) < kTinyW ? kTinyW : w;
+                        s_w[g] = valid ? w : (g == 0 ? wprev : s_w[g - 1]);
+                        s_sp[g] = sp2;
+                        s_q[g] = CHAIN ? ex2(sp2 * a_l[0]) : 1.f;
+                        s_du[g] = dskip * uv;
+                        s_g[g] = 1.f;
                         if (GATE) {
-                            const float zv = Io<io_t>::ld(sz + r * DC + tid);
-                            y *= zv * rcp(1.f + ex2(-zv * kLog2e));
+                            const float zv = Io<io_t>::ld(sz + (r ^ xmask) * DC + tid);
+                            s_g[g] = zv * rcp(1.f + ex2(-zv * kLog2e));
                         }
-                        static_cast<io_t*>(p.out)[(b * p.L + pp) * p.D + d] = Io<io_t>::st(y);
                     }
+#pragma unroll
+                    for (int g = 0; g < kGroup; ++g)
+                        s_rr[g] = (g == 0 ? wprev : s_w[g - 1]) * rcp(s_w[g]);
+                    wprev = s_w[kGroup - 1];
+#pragma unroll
+                    for (int g = 0; g < kGroup; ++g) {
+                        const int r = r0 + g;  // < kTile; rows past the tile end read B = C = 0
+                        const float rr = s_rr[g];
+                        if (PHASE1)
+                            dsum += s_sp[g];
+                        // c[n] = (w_prev/w) * exp(Delta*A[d,n]) as pairs (n, n+1)
+                        float2 cp[NS / 2];
+                        if (CHAIN) {
+                            // q^(n+1) by a tree of depth log2(N): pair j = pair (j-m) * q^(2m)
+                            const float q = s_q[g];
+                            float qm = q * q;
+                            cp[0] = make_float2(rr * q, rr * qm);
+#pragma unroll
+                            for (int m = 1; m < NS / 2; m *= 2) {
+                                const float2 qq = make_float2(qm, qm);
+#pragma unroll
+                                for (int j = m; j < 2 * m && j < NS / 2; ++j)
+                                    cp[j] = __fmul2_rn(cp[j - m], qq);
+                                qm = qm * qm;
+                            }
+                        } else {
+                            const float sp2 = s_sp[g];
+#pragma unroll
+                            for (int j = 0; j < NS / 2; ++j)
+                                cp[j] = make_float2(rr * ex2(sp2 * a_l[2 * j]),
+                                                    rr * ex2(sp2 * a_l[2 * j + 1]));
+                        }
+                        float2 yacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                          make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+                        for (int n4 = 0; n4 < NS / 4; ++n4) {
+                            const float4 bq = B4[r * (NS / 4) + n4];
+                            kst2[2 * n4] =
+                                __ffma2_rn(cp[2 * n4], kst2[2 * n4], make_float2(bq.x, bq.y));
+                            kst2[2 * n4 + 1] = __ffma2_rn(cp[2 * n4 + 1], kst2[2 * n4 + 1],
+                                                          make_float2(bq.z, bq.w));
+                            if (!PHASE1) {
+                                const float4 cq = C4[r * (NS / 4) + n4];
+                                yacc[(2 * n4) & 3] = __ffma2_rn(make_float2(cq.x, cq.y),
+                                                                kst2[2 * n4], yacc[(2 * n4) & 3]);
+                                yacc[(2 * n4 + 1) & 3] =
+                                    __ffma2_rn(make_float2(cq.z, cq.w), kst2[2 * n4 + 1],
+                                               yacc[(2 * n4 + 1) & 3]);
+                            }
+                        }
+                        if (!PHASE1) {
+                            const float2 ys = __fadd2_rn(__fadd2_rn(yacc[0], yacc[1]),
+                                                         __fadd2_rn(yacc[2], yacc[3]));
+                            float y = fmaf(s_w[g], ys.x + ys.y, s_du[g]);
+                            if (r < rows) {
+                                if (YPART) {
+                                    p.ypart[orow[r] + tid] = y;
+                                } else {
+                                    if (GATE)
+                                        y *= s_g[g];
+                                    static_cast<io_t*>(p.out)[orow[r] + tid] = Io<io_t>::st(y);
+                                }
+                            }
+                        }
+                    }
+                };
+                for (int r0 = 0; r0 < rows; r0 += kGroup) {
+                    if (use_chain)
+                        group(std::true_type{}, r0);
+                    else
+                        group(std::false_type{}, r0);
                 }
             }
         }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&empty[st]);
     }
 
-    if (failed_at >= 0) {
-        // let the copies this CTA still has in flight (tiles failed_at .. issued-1) land before
-        // its shared memory goes away; each wait is bounded as well
+    if (failed) {
+        // let the copies this CTA has in flight land before its shared memory goes away; the
+        // waits are bounded as well
         if (warp == 0 && lane == 0) {
-            for (int64_t j = failed_at; j < issued; ++j)
+            for (int64_t j = 0; j < issued; ++j)
                 (void)mbar_wait_bounded(&full[j % kStages], static_cast<uint32_t>((j / kStages) & 1),
-                                        kWaitLimitNs / 4);
+                                        kWaitLimitNs / 8);
         }
-        __syncthreads();
         return;
     }
 
@@ -539,12 +765,76 @@ __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ Merg
 
 constexpr int kWarps = 2;
 
-template <typename io_t, int NS, bool GATE, bool PHASE1>
-cudaError_t launch_t(const ScanParams& p, cudaStream_t stream)
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link-time libcuda dependency).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }();
+    return fn;
+}
+
+// A row-major tensor of `rank` dims (innermost first) with element strides `pitch` bytes for
+// dims 1.., read in boxes `box`; out-of-range elements read as zero.
+bool encode(CUtensorMap* map, const void* base, bool bf16, int rank, const cuuint64_t* dims,
+            const cuuint64_t* pitch, const cuuint32_t* box)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn)
+        return false;
+    const cuuint32_t unit[3] = {1, 1, 1};
+    return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+              static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, pitch, box, unit,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename io_t>
+cudaError_t make_maps(ScanParams& p, bool need_z)
+{
+    constexpr bool bf16 = sizeof(io_t) == 2;
+    const cuuint64_t esz = sizeof(io_t);
+    const cuuint64_t D = static_cast<cuuint64_t>(p.D);
+    const cuuint32_t box2[2] = {static_cast<cuuint32_t>(32 * kWarps), static_cast<cuuint32_t>(kTile)};
+    const cuuint64_t pitch2[1] = {D * esz};
+    const cuuint64_t dims_bl[2] = {D, static_cast<cuuint64_t>(p.batch * p.L)};
+    const cuuint64_t dims_kbl[2] = {D, static_cast<cuuint64_t>(p.K * p.batch * p.L)};
+    if (!encode(&p.tm_u, p.u, bf16, 2, dims_bl, pitch2, box2) ||
+        !encode(&p.tm_dl, p.delta, bf16, 2, dims_kbl, pitch2, box2) ||
+        (need_z && !encode(&p.tm_z, p.z, bf16, 2, dims_bl, pitch2, box2)))
+        return cudaErrorInvalidValue;
+    bool col = false;
+    for (int k = 0; k < p.K; ++k)
+        col = col || p.dirs[k] == SS_DIR_COL || p.dirs[k] == SS_DIR_COL_REV;
+    p.col3d = (col && p.H > 0 && p.H % 8 == 0) ? 1 : 0;
+    if (p.col3d) {
+        const cuuint32_t box3[3] = {static_cast<cuuint32_t>(32 * kWarps), 1, 8};
+        const cuuint64_t pitch3[2] = {D * esz, static_cast<cuuint64_t>(p.W) * D * esz};
+        const cuuint64_t dims3[3] = {D, static_cast<cuuint64_t>(p.W),
+                                     static_cast<cuuint64_t>(p.batch * p.H)};
+        if (!encode(&p.tm_u3, p.u, bf16, 3, dims3, pitch3, box3) ||
+            (need_z && !encode(&p.tm_z3, p.z, bf16, 3, dims3, pitch3, box3)))
+            return cudaErrorInvalidValue;
+    }
+    return cudaSuccess;
+}
+
+template <typename io_t, int NS, bool GATE, bool PHASE1, bool YPART>
+cudaError_t launch_t(const ScanParams& p0, cudaStream_t stream)
 {
     using Lay = Layout<io_t, NS, kWarps, GATE, PHASE1>;
-    auto kern = scan_kernel<io_t, NS, kWarps, GATE, PHASE1>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::BYTES);
+    auto kern = scan_kernel<io_t, NS, kWarps, GATE, PHASE1, YPART>;
+    ScanParams p = p0;
+    cudaError_t e = make_maps<io_t>(p, Lay::HAS_Z);
+    if (e != cudaSuccess)
+        return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::BYTES);
     if (e != cudaSuccess)
         return e;
     const int64_t ntiles = (p.D + Lay::DC - 1) / Lay::DC;
@@ -559,11 +849,12 @@ cudaError_t launch_t(const ScanParams& p, cudaStream_t stream)
 template <typename io_t, int NS>
 cudaError_t launch_ns(const ScanParams& p, int phase1, cudaStream_t stream)
 {
-    const bool gate = p.z != nullptr && p.ypart == nullptr;
     if (phase1)
-        return launch_t<io_t, NS, false, true>(p, stream);
-    return gate ? launch_t<io_t, NS, true, false>(p, stream)
-                : launch_t<io_t, NS, false, false>(p, stream);
+        return launch_t<io_t, NS, false, true, false>(p, stream);
+    if (p.ypart)
+        return launch_t<io_t, NS, false, false, true>(p, stream);
+    return p.z ? launch_t<io_t, NS, true, false, false>(p, stream)
+               : launch_t<io_t, NS, false, false, false>(p, stream);
 }
 
 template <typename io_t>
