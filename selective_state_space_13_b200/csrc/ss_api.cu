@@ -10,9 +10,11 @@
 namespace {
 
 constexpr int64_t kMaxSeqlen = (int64_t{1} << 31) - 1;
-// Auto segment choice: split sequences until about this many CTAs exist (4 per SM on B200),
-// but never below this many steps per segment.
-constexpr int64_t kTargetCtas = 4 * 148;
+// Automatic segment choice (measured on B200): when the (direction, batch row, channel tile)
+// units give fewer than about 3 CTAs per SM, split each sequence until they do, and split long
+// sequences into segments of about kLongSegSteps steps; never below kMinSegSteps steps.
+constexpr int64_t kTargetCtas = 3 * 148;
+constexpr int64_t kLongSegSteps = 4096;
 constexpr int64_t kMinSegSteps = 16 * ss::kTile;
 constexpr int kMaxSegments = 1024;
 
@@ -113,8 +115,11 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
         const int64_t ctas = ((pl->D + ss::channels_per_cta() - 1) / ss::channels_per_cta()) *
                              pl->batch * pl->K;
         seg = 1;
-        if (ctas > 0 && ctas < kTargetCtas / 2) {
+        if (ctas > 0 && ctas < kTargetCtas) {
             int64_t want = (kTargetCtas + ctas - 1) / ctas;
+            const int64_t by_len = L / kLongSegSteps;
+            if (want < by_len)
+                want = by_len;
             const int64_t cap = L / kMinSegSteps;
             if (want > cap)
                 want = cap;

@@ -498,14 +498,29 @@ __global__ void __launch_bounds__(32 * WARPS)
     }
     float dsum = 0.f;  // sum of Delta*log2(e) over this segment (aggregate launch)
 
-    // ---- prologue: warp 0 fills the first kStages-2 stages
-    int64_t issued = 0;
-    if (warp == 0)
-        for (; issued < kStages - 2 && issued < ntile_t; ++issued)
-            issue(issued);
-
+    // ---- pipeline.  Producer duty rotates: in iteration `it`, warp it % WARPS converts the B/C
+    // of tile it+1 (one tile ahead, so no warp waits for a conversion) and refills the stage
+    // released by tile it-2 with tile it+kStages-2.  Warp 0 starts the pipeline.
+    volatile int* s_issued = s_abort + 1;  // tiles issued so far (read only on the error path)
     bool failed = false;
-    for (int64_t it = 0; it < ntile_t; ++it) {
+    int64_t my_issued = 0;                 // tiles this warp has issued (error path)
+    if (warp == 0) {
+        int64_t j = 0;
+        for (; j < kStages - 2 && j < ntile_t; ++j)
+            issue(j);
+        my_issued = j;
+        if (lane == 0)
+            *s_issued = static_cast<int>(j);
+        if (!mbar_wait_bounded(&full[0], 0, kWaitLimitNs)) {
+            failed = true;
+        } else {
+            convert(0);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&ready[0]);
+        }
+    }
+    for (int64_t it = 0; it < ntile_t && !failed; ++it) {
         const int st = static_cast<int>(it % kStages);
         const uint32_t ph = static_cast<uint32_t>((it / kStages) & 1);
         unsigned char* sb = smem + st * Lay::STAGE;
@@ -514,32 +529,37 @@ __global__ void __launch_bounds__(32 * WARPS)
             failed = true;
             break;
         }
-        if (warp == 0) {
-            if (!mbar_wait_bounded(&full[st], ph, kWaitLimitNs)) {
-                failed = true;
-            } else {
-                convert(it);
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&ready[st]);
-                // refill the stage released two tiles ago
-                const int64_t nx = it + kStages - 2;
-                if (nx < ntile_t) {
-                    if (nx >= kStages &&
-                        !mbar_wait_bounded(&empty[nx % kStages],
-                                           static_cast<uint32_t>(((nx / kStages) - 1) & 1),
-                                           kWaitLimitNs))
-                        failed = true;
-                    else
-                        issue(nx);
-                    issued = nx + 1;
+        if (warp == static_cast<int>(it % WARPS)) {
+            const int64_t n1 = it + 1;
+            if (n1 < ntile_t) {
+                if (!mbar_wait_bounded(&full[n1 % kStages],
+                                       static_cast<uint32_t>((n1 / kStages) & 1), kWaitLimitNs)) {
+                    failed = true;
+                } else {
+                    convert(n1);
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&ready[n1 % kStages]);
                 }
             }
-        } else {
-            if (!mbar_wait_bounded(&ready[st], ph, kWaitLimitNs) ||
-                !mbar_wait_bounded(&full[st], ph, kWaitLimitNs))
-                failed = true;
+            const int64_t nx = it + kStages - 2;
+            if (!failed && nx < ntile_t) {
+                if (nx >= kStages &&
+                    !mbar_wait_bounded(&empty[nx % kStages],
+                                       static_cast<uint32_t>(((nx / kStages) - 1) & 1),
+                                       kWaitLimitNs)) {
+                    failed = true;
+                } else {
+                    issue(nx);
+                    my_issued = nx + 1;
+                    if (lane == 0)
+                        *s_issued = static_cast<int>(nx + 1);
+                }
+            }
         }
+        if (!failed && !(mbar_wait_bounded(&ready[st], ph, kWaitLimitNs) &&
+                         mbar_wait_bounded(&full[st], ph, kWaitLimitNs)))
+            failed = true;
         if (failed) {
             atomicOr(&g_ss_status, kStatusTimeout);
             *s_abort = 1;
@@ -713,12 +733,17 @@ __global__ void __launch_bounds__(32 * WARPS)
     }
 
     if (failed) {
-        // let the copies this CTA has in flight land before its shared memory goes away; the
+        atomicOr(&g_ss_status, kStatusTimeout);
+        *s_abort = 1;
+        // let the copies this warp issued land before the CTA's shared memory goes away; the
         // waits are bounded as well
-        if (warp == 0 && lane == 0) {
-            for (int64_t j = 0; j < issued; ++j)
-                (void)mbar_wait_bounded(&full[j % kStages], static_cast<uint32_t>((j / kStages) & 1),
-                                        kWaitLimitNs / 8);
+        if (lane == 0) {
+            for (int64_t j = 0; j < my_issued; ++j) {
+                const int issuer = j < kStages - 2 ? 0 : static_cast<int>((j - (kStages - 2)) % WARPS);
+                if (issuer == warp)
+                    (void)mbar_wait_bounded(&full[j % kStages],
+                                            static_cast<uint32_t>((j / kStages) & 1), kWaitLimitNs / 8);
+            }
         }
         return;
     }
