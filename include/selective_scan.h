@@ -59,7 +59,9 @@ typedef enum {
     SS_ERR_UNSUPPORTED = 6,   /* dstate > SS_MAX_DSTATE or an unsupported option               */
     SS_ERR_CUDA = 7,          /* the CUDA runtime reported an error at launch                  */
     SS_ERR_WORKSPACE = 8,     /* workspace NULL or smaller than selective_scan_workspace_size  */
-    SS_ERR_DEVICE_TIMEOUT = 9 /* a kernel gave up a bounded wait (reported by device_status)   */
+    SS_ERR_DEVICE_TIMEOUT = 9, /* a kernel gave up a bounded wait (reported by device_status)  */
+    SS_ERR_SCRATCH_LIMIT = 10  /* selective_scan_fwd_noalloc: the problem needs more scratch than
+                                  SS_NOALLOC_SCRATCH_BYTES                                      */
 } ss_status;
 
 typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_dtype;
@@ -146,6 +148,41 @@ int64_t ss_direction_position(const ss_direction_map* dmap, int32_t k, int64_t L
  * the current device gave up a bounded wait since the last call with clear != 0 (SS_OK
  * otherwise, SS_ERR_CUDA if the runtime failed).  With clear != 0 the flag is reset. */
 ss_status selective_scan_device_status(void* stream, int32_t clear);
+
+/* Bytes of the fixed scratch array that selective_scan_fwd_noalloc uses (16 MiB). */
+#define SS_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * selective_scan_fwd_noalloc -- the same scan as selective_scan_fwd, for callers that cannot
+ * allocate device memory.  (The pages have no counterpart to this entry point; it exists for
+ * deployments, not for the method.)
+ *
+ * Who needs it: callers whose device memory is fixed when they start -- a plugin inside a host
+ * application that owns the allocator, an inference server that sizes one arena up front, or a
+ * latency-critical loop that must not call cudaMalloc (which can synchronise the device) -- and
+ * that therefore cannot provide the workspace selective_scan_fwd asks for.
+ *
+ * Arguments are those of selective_scan_fwd without `workspace` / `workspace_bytes`; the caller
+ * still passes every input and output.  The scratch comes from one array of this library's
+ * device memory of SS_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the library holds
+ * until the process exits.  The call allocates nothing (no cudaMalloc, no cudaFree, no
+ * allocating library routine).
+ *   - A problem whose selective_scan_workspace_size() exceeds SS_NOALLOC_SCRATCH_BYTES is
+ *     rejected with SS_ERR_SCRATCH_LIMIT before anything runs (at the default options: m130
+ *     and the 131072-step sequence fit; the Vim and SS2D workloads, whose per-direction
+ *     outputs need far more, do not).
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current); make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents.  Nothing in it has to
+ *     start at zero: every value a call reads from it was written earlier by the same call.
+ *     Calls whose work overlaps on the GPU (other streams, other host threads) race on the
+ *     array; order them, for example on one stream.
+ */
+ss_status selective_scan_fwd_noalloc(const ss_shape* shape, const void* u, const void* delta,
+                                     const float* A, const void* B, const void* C,
+                                     const float* Dskip, const void* z, const float* delta_bias,
+                                     int32_t softplus, const ss_direction_map* dmap, void* out,
+                                     float* last_state, void* stream, const ss_launch_opts* opts);
 
 /* Human-readable name of a status code (static storage). */
 const char* ss_status_str(ss_status status);

@@ -303,6 +303,8 @@ const char* ss_status_str(ss_status status)
     case SS_ERR_CUDA: return "SS_ERR_CUDA: the CUDA runtime reported an error";
     case SS_ERR_WORKSPACE: return "SS_ERR_WORKSPACE: workspace missing or too small";
     case SS_ERR_DEVICE_TIMEOUT: return "SS_ERR_DEVICE_TIMEOUT: a kernel gave up a bounded wait";
+    case SS_ERR_SCRATCH_LIMIT:
+        return "SS_ERR_SCRATCH_LIMIT: the problem needs more scratch than SS_NOALLOC_SCRATCH_BYTES";
     }
     return "unknown ss_status";
 }

@@ -19,6 +19,7 @@ import threading
 from . import build as _build
 
 SS_OK = 0
+SS_ERR_SCRATCH_LIMIT = 10
 SS_F32, SS_BF16 = 0, 1
 SS_DIR_FWD, SS_DIR_REV, SS_DIR_COL, SS_DIR_COL_REV = 0, 1, 2, 3
 SS_FLAG_GENERIC_A = 1
@@ -27,10 +28,12 @@ SS_MAX_DIRS = 4
 
 STATUS_NAMES = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE",
                 4: "SS_ERR_ALIGN", 5: "SS_ERR_DIRMAP", 6: "SS_ERR_UNSUPPORTED", 7: "SS_ERR_CUDA",
-                8: "SS_ERR_WORKSPACE", 9: "SS_ERR_DEVICE_TIMEOUT"}
+                8: "SS_ERR_WORKSPACE", 9: "SS_ERR_DEVICE_TIMEOUT", 10: "SS_ERR_SCRATCH_LIMIT"}
+SS_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 EXPORTED = ("selective_scan_workspace_size", "selective_scan_fwd", "ss_direction_position",
-            "selective_scan_device_status", "ss_status_str", "ss_abi_version")
+            "selective_scan_device_status", "ss_status_str", "ss_abi_version",
+            "selective_scan_fwd_noalloc")
 
 
 class SsShape(ctypes.Structure):
@@ -114,6 +117,10 @@ def load():
         lib.ss_status_str.argtypes = [ctypes.c_int]
         lib.ss_abi_version.restype = i32
         lib.ss_abi_version.argtypes = []
+        lib.selective_scan_fwd_noalloc.restype = ctypes.c_int
+        lib.selective_scan_fwd_noalloc.argtypes = [ctypes.POINTER(SsShape), vp, vp, vp, vp, vp, vp,
+                                                   vp, vp, i32, ctypes.POINTER(SsDirectionMap), vp,
+                                                   vp, vp, ctypes.POINTER(SsLaunchOpts)]
         _lib = lib
         return lib
 
@@ -188,6 +195,18 @@ def selective_scan_fwd_raw(shape: SsShape, u, delta, A, B, C, Dskip, z, delta_bi
         ctypes.byref(dmap) if dmap is not None else None, out or None, last_state or None,
         workspace or None, int(workspace_bytes), stream or None,
         ctypes.byref(opts) if opts is not None else None))
+
+
+def selective_scan_fwd_noalloc_raw(shape: SsShape, u, delta, A, B, C, Dskip, z, delta_bias,
+                                   softplus, dmap, out, last_state, stream, opts=None) -> int:
+    """selective_scan_fwd_noalloc with integer device addresses (0 = NULL); returns the
+    ss_status.  For callers that cannot allocate device memory: the scratch is the library's own
+    fixed array (SS_NOALLOC_SCRATCH_BYTES), shared by all calls."""
+    return int(load().selective_scan_fwd_noalloc(
+        ctypes.byref(shape), u or None, delta or None, A or None, B or None, C or None,
+        Dskip or None, z or None, delta_bias or None, int(bool(softplus)),
+        ctypes.byref(dmap) if dmap is not None else None, out or None, last_state or None,
+        stream or None, ctypes.byref(opts) if opts is not None else None))
 
 
 # ----------------------------------------------------------------------------- torch front end
