@@ -162,6 +162,15 @@ class ClockSampler:
                 "samples": len(self.samples), "source": "NVML during the timed region"}
 
 
+def workload_of(args) -> wl.Workload:
+    w = wl.WORKLOADS[args.workload]
+    if args.seqlen:
+        if w.H:
+            raise SystemExit("--seqlen does not apply to image workloads")
+        w = wl.variant(w.name, seqlen=args.seqlen)
+    return w
+
+
 def workload_bytes(w: wl.Workload) -> int:
     return w.algorithmic_bytes(with_last_state=w.name in RETURNS_LAST_STATE)
 
@@ -198,7 +207,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
-    w = wl.WORKLOADS[args.workload]
+    w = workload_of(args)
     inp = wl.make_inputs(w)
     threads = oracle.max_threads()
     # each step: the oracle on a channel sample worth about 2e7 state updates
@@ -241,7 +250,7 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
-    w = wl.WORKLOADS[args.workload]
+    w = workload_of(args)
     inp = wl.make_inputs(w)
     t = to_device(inp, device)
     want_last = w.name in RETURNS_LAST_STATE
@@ -370,7 +379,9 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == wl.BF16 else "f32",
         "data": "synthetic (seeded N(0,1) inputs, A=-(n+1), log-uniform Delta bias)",
-        "config": {"workload": wl.DESCRIPTIONS[w.name], "name": w.name, "batch": w.batch,
+        "config": {"workload": wl.DESCRIPTIONS[w.name] + (
+                       " (seqlen overridden to %d)" % w.seqlen if args.seqlen else ""),
+                   "name": w.name, "batch": w.batch,
                    "seqlen": w.seqlen, "dim": w.dim, "dstate": w.dstate, "directions": w.K,
                    "gate": w.gate, "returns_last_state": want_last,
                    "parallelism": "independent problems per rank" if world > 1 else "1 GPU",
@@ -406,6 +417,8 @@ def parse(argv=None):
     ap.add_argument("--workload", choices=sorted(wl.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--segments", type=int, default=0, help="0 = the library's choice")
     ap.add_argument("--flags", type=int, default=0, help="SS_FLAG_* bits (1 = generic A)")
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="override the workload's sequence length (smaller cases for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-updates", type=float, default=4e9,
