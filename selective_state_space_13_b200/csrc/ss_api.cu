@@ -11,8 +11,11 @@ namespace {
 
 constexpr int64_t kMaxSeqlen = (int64_t{1} << 31) - 1;
 // Automatic segment choice (measured on B200): when the (direction, batch row, channel tile)
-// units give fewer than about 3 CTAs per SM, split each sequence until they do, and split long
-// sequences into segments of about kLongSegSteps steps; never below kMinSegSteps steps.
+// units give fewer than about 1.5 CTAs per SM, split each sequence until they reach about 3 per
+// SM, and split long sequences into segments of about kLongSegSteps steps; never below
+// kMinSegSteps steps.  (With more units, the segment-aggregate launch costs more than the
+// parallelism it adds.)
+constexpr int64_t kSplitBelowCtas = 222;
 constexpr int64_t kTargetCtas = 3 * 148;
 constexpr int64_t kLongSegSteps = 4096;
 constexpr int64_t kMinSegSteps = 16 * ss::kTile;
@@ -115,7 +118,7 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
         const int64_t ctas = ((pl->D + ss::channels_per_cta() - 1) / ss::channels_per_cta()) *
                              pl->batch * pl->K;
         seg = 1;
-        if (ctas > 0 && ctas < kTargetCtas) {
+        if (ctas > 0 && ctas < kSplitBelowCtas) {
             int64_t want = (kTargetCtas + ctas - 1) / ctas;
             const int64_t by_len = L / kLongSegSteps;
             if (want < by_len)

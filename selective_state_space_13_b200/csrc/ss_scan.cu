@@ -446,6 +446,30 @@ __global__ void __launch_bounds__(32 * WARPS)
         const io_t* cr = reinterpret_cast<const io_t*>(sb + Lay::OFF_CR) + cskip;
         float* bf = reinterpret_cast<float*>(sb + Lay::OFF_BF);
         const float bscale = PRECISE ? 1.f : kLn2;
+        if (!PRECISE && NS == 16 && p.N == 16 && bskip == 0 && cskip == 0) {
+            // 16 bf16 rows of 16 values per tensor: lane l converts 8 values (16 bytes) of B and
+            // 8 of C; rows past the tile's end become 0
+            static_assert(kTile * 16 * 2 == 32 * 16, "one 16-byte chunk per lane and tensor");
+            const int r = lane >> 1;
+            const bool ok = r < rows;
+            auto cvt8 = [&](const io_t* src, float* dst, float scale) {
+                const uint4 w = *reinterpret_cast<const uint4*>(src + 8 * lane);
+                const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    f[2 * i] = ok ? __uint_as_float(v[i] << 16) * scale : 0.f;
+                    f[2 * i + 1] = ok ? __uint_as_float(v[i] & 0xffff0000u) * scale : 0.f;
+                }
+                float4* d4 = reinterpret_cast<float4*>(dst + 8 * lane);
+                d4[0] = make_float4(f[0], f[1], f[2], f[3]);
+                d4[1] = make_float4(f[4], f[5], f[6], f[7]);
+            };
+            cvt8(br, bf, bscale);
+            if (Lay::HAS_C)
+                cvt8(cr, bf + kTile * NS, 1.f);
+            return;
+        }
         for (int idx = lane; idx < kTile * NS; idx += 32) {
             const int r = idx / NS, n = idx - (idx / NS) * NS;
             const bool ok = r < rows && n < p.N;
@@ -768,21 +792,60 @@ __global__ void __launch_bounds__(32 * WARPS)
 
 // ---------------------------------------------------------------------------- merge kernel
 
-template <typename io_t, bool GATE>
+// Four adjacent channels per thread: 16-byte fp32 loads from every direction's plane, all issued
+// before the sum; the partial outputs are read once, so loads and stores stream past L1/L2.
+template <typename io_t> struct Io4;
+template <> struct Io4<float> {
+    static __device__ __forceinline__ float4 ld(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
+    static __device__ __forceinline__ void st(float* p, float4 v) { __stcs(reinterpret_cast<float4*>(p), v); }
+};
+template <> struct Io4<__nv_bfloat16> {
+    static __device__ __forceinline__ float4 ld(const __nv_bfloat16* p)
+    {
+        const uint2 w = __ldcs(reinterpret_cast<const uint2*>(p));
+        return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                           __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+    }
+    static __device__ __forceinline__ void st(__nv_bfloat16* p, float4 v)
+    {
+        const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+        const __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+        uint2 w;
+        w.x = *reinterpret_cast<const uint32_t*>(&a);
+        w.y = *reinterpret_cast<const uint32_t*>(&b);
+        __stcs(reinterpret_cast<uint2*>(p), w);
+    }
+};
+
+__device__ __forceinline__ float silu_f(float z) { return z * rcp(1.f + ex2(-z * kLog2e)); }
+
+template <typename io_t, bool GATE, int K>
 __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ MergeParams p)
 {
-    const int64_t total = p.rows * p.D;
-    const int64_t plane = total;
-    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+    const int64_t plane = p.rows * p.D;
+    const int64_t n4 = plane / 4;  // D is a multiple of 4
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        float y = 0.f;
-        for (int k = 0; k < p.K; ++k)
-            y += p.ypart[k * plane + i];
-        if (GATE) {
-            const float zv = Io<io_t>::ld(static_cast<const io_t*>(p.z) + i);
-            y *= zv * rcp(1.f + ex2(-zv * kLog2e));
+        float4 part[K];
+#pragma unroll
+        for (int k = 0; k < K; ++k)
+            part[k] = Io4<float>::ld(p.ypart + k * plane + 4 * i);
+        float4 y = part[0];
+#pragma unroll
+        for (int k = 1; k < K; ++k) {
+            y.x += part[k].x;
+            y.y += part[k].y;
+            y.z += part[k].z;
+            y.w += part[k].w;
         }
-        static_cast<io_t*>(p.out)[i] = Io<io_t>::st(y);
+        if (GATE) {
+            const float4 zv = Io4<io_t>::ld(static_cast<const io_t*>(p.z) + 4 * i);
+            y.x *= silu_f(zv.x);
+            y.y *= silu_f(zv.y);
+            y.z *= silu_f(zv.z);
+            y.w *= silu_f(zv.w);
+        }
+        Io4<io_t>::st(static_cast<io_t*>(p.out) + 4 * i, y);
     }
 }
 
@@ -902,29 +965,33 @@ cudaError_t launch_scan(const ScanParams& p, int io_dtype, int phase1, cudaStrea
                                : launch_io<float>(p, phase1, stream);
 }
 
+template <typename io_t, bool GATE>
+void merge_k(const MergeParams& p, unsigned blocks, cudaStream_t stream)
+{
+    switch (p.K) {
+    case 2: merge_kernel<io_t, GATE, 2><<<blocks, 256, 0, stream>>>(p); break;
+    case 3: merge_kernel<io_t, GATE, 3><<<blocks, 256, 0, stream>>>(p); break;
+    default: merge_kernel<io_t, GATE, 4><<<blocks, 256, 0, stream>>>(p); break;
+    }
+}
+
 cudaError_t launch_merge(const MergeParams& p, int io_dtype, cudaStream_t stream)
 {
-    const int64_t total = p.rows * p.D;
-    if (total <= 0)
+    const int64_t n4 = p.rows * p.D / 4;
+    if (n4 <= 0)
         return cudaSuccess;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int64_t blocks = (total + 255) / 256;
-    if (blocks > static_cast<int64_t>(sms) * 16)
-        blocks = static_cast<int64_t>(sms) * 16;
+    int64_t blocks = (n4 + 255) / 256;
+    if (blocks > static_cast<int64_t>(sms) * 8)
+        blocks = static_cast<int64_t>(sms) * 8;
+    const unsigned nb = static_cast<unsigned>(blocks);
     const bool gate = p.z != nullptr;
-    if (io_dtype == SS_BF16) {
-        if (gate)
-            merge_kernel<__nv_bfloat16, true><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
-        else
-            merge_kernel<__nv_bfloat16, false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
-    } else {
-        if (gate)
-            merge_kernel<float, true><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
-        else
-            merge_kernel<float, false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
-    }
+    if (io_dtype == SS_BF16)
+        gate ? merge_k<__nv_bfloat16, true>(p, nb, stream) : merge_k<__nv_bfloat16, false>(p, nb, stream);
+    else
+        gate ? merge_k<float, true>(p, nb, stream) : merge_k<float, false>(p, nb, stream);
     return cudaGetLastError();
 }
 
