@@ -11,12 +11,12 @@ namespace {
 
 constexpr int64_t kMaxSeqlen = (int64_t{1} << 31) - 1;
 // Automatic segment choice (measured on B200): when the (direction, batch row, channel tile)
-// units give fewer than about 1.5 CTAs per SM, split each sequence until they reach about 3 per
+// units give fewer than about 1.5 CTAs per SM, split each sequence until they reach about 4 per
 // SM, and split long sequences into segments of about kLongSegSteps steps; never below
 // kMinSegSteps steps.  (With more units, the segment-aggregate launch costs more than the
 // parallelism it adds.)
 constexpr int64_t kSplitBelowCtas = 222;
-constexpr int64_t kTargetCtas = 3 * 148;
+constexpr int64_t kTargetCtas = 4 * 148;
 constexpr int64_t kLongSegSteps = 4096;
 constexpr int64_t kMinSegSteps = 16 * ss::kTile;
 constexpr int kMaxSegments = 1024;

@@ -11,9 +11,8 @@
 
 namespace ss {
 
-// Steps per pipeline stage and number of stages of the shared-memory ring.
+// Steps per pipeline stage of the shared-memory ring.
 constexpr int kTile = 16;
-constexpr int kStages = 5;
 // Rows whose per-step scalars the fast path computes together.
 constexpr int kGroup = 8;
 

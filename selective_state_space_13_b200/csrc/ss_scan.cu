@@ -4,7 +4,7 @@
 // N-state vector in registers for the whole segment ("Understanding Mamba from zero" sec. 5:
 // per channel and per state the recurrence is the scalar affine map h_t = a_t h_{t-1} + b_t).
 // A CTA of 32*WARPS threads owns a tile of adjacent channels.  Its inputs stream through a
-// ring of kStages shared-memory stages of kTile steps each; warp 0 fills the ring with bulk
+// ring of 4-5 shared-memory stages of kTile steps each; warp 0 fills the ring with bulk
 // asynchronous copies (TMA, cp.async.bulk) that complete on an mbarrier, one copy per row of
 // u / z (rows picked through the direction's index map) and delta (scan order), plus one copy
 // each for the B and C tiles, which every channel of the CTA shares.  B and C are converted to
@@ -167,6 +167,13 @@ __device__ __forceinline__ float lg2(float x)
     return y;
 }
 
+__device__ __forceinline__ float tanh_approx(float x)
+{
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ float rcp(float x)
 {
     float y;
@@ -245,7 +252,7 @@ __host__ __device__ __forceinline__ int64_t position(int32_t dir, int64_t L, int
 
 // One pipeline stage holds kTile rows of u, delta and z for the CTA's channels (as copied),
 // the raw B and C tiles, their fp32 copies, and the output row offsets of the tile.
-template <typename io_t, int NS, int WARPS, bool GATE, bool PHASE1>
+template <typename io_t, int NS, int WARPS, bool GATE, bool PHASE1, int STAGES>
 struct Layout {
     static constexpr int DC = 32 * WARPS;                           // channels per CTA
     static constexpr int ROW = DC * (int)sizeof(io_t);               // bytes of one row slice
@@ -253,20 +260,24 @@ struct Layout {
     static constexpr int BCRAW = ((kTile * NS * (int)sizeof(io_t) + 32 + 15) / 16) * 16;
     static constexpr bool HAS_Z = GATE && !PHASE1;
     static constexpr bool HAS_C = !PHASE1;
+    // each field is an array over the stages; tile fields come first (128-byte aligned for the
+    // tensor copies), the rest is packed at 16-byte alignment to keep the CTA's footprint small
     static constexpr int OFF_U = 0;
-    static constexpr int OFF_DL = OFF_U + ROWS;
-    static constexpr int OFF_Z = OFF_DL + ROWS;
-    static constexpr int OFF_BR = OFF_Z + (HAS_Z ? ROWS : 0);
-    static constexpr int OFF_CR = OFF_BR + BCRAW;
-    static constexpr int OFF_BF = OFF_CR + (HAS_C ? BCRAW : 0);      // fp32 B, then fp32 C
+    static constexpr int OFF_DL = OFF_U + STAGES * ROWS;
+    static constexpr int OFF_Z = OFF_DL + STAGES * ROWS;
+    static constexpr int OFF_BR = OFF_Z + (HAS_Z ? STAGES * ROWS : 0);
+    static constexpr int OFF_CR = OFF_BR + STAGES * BCRAW;
+    static constexpr int OFF_BF = OFF_CR + (HAS_C ? STAGES * BCRAW : 0);  // fp32 B, then fp32 C
     static constexpr int BF_ONE = kTile * NS * 4;
-    static constexpr int OFF_OUT = OFF_BF + BF_ONE * (HAS_C ? 2 : 1);  // int64 row offsets
-    static constexpr int STAGE = ((OFF_OUT + kTile * 8 + 127) / 128) * 128;
-    static constexpr int OFF_BAR = kStages * STAGE;                  // full, ready, empty
-    static constexpr int OFF_FLAG = OFF_BAR + 3 * kStages * 8;
+    static constexpr int BF_STRIDE = BF_ONE * (HAS_C ? 2 : 1);
+    static constexpr int OFF_OUT = OFF_BF + STAGES * BF_STRIDE;           // int64 row offsets
+    static constexpr int OUT_STRIDE = kTile * 8;
+    static constexpr int OFF_BAR = OFF_OUT + STAGES * OUT_STRIDE;         // full, ready, empty
+    static constexpr int OFF_FLAG = OFF_BAR + 3 * STAGES * 8;
     static constexpr int BYTES = OFF_FLAG + 16;
-    static_assert(ROW % 16 == 0 && BCRAW % 16 == 0 && OFF_BF % 16 == 0 && OFF_OUT % 8 == 0,
-                  "TMA destinations and vector accesses need 16-byte alignment");
+    static_assert(ROWS % 128 == 0 && BCRAW % 16 == 0 && OFF_BR % 128 == 0 && OFF_BF % 16 == 0 &&
+                      BF_STRIDE % 16 == 0 && OFF_OUT % 8 == 0,
+                  "tensor-copy destinations need 128-byte and vector accesses 16-byte alignment");
 };
 
 // ---------------------------------------------------------------------------- the scan kernel
@@ -282,7 +293,14 @@ template <typename io_t, int NS, int WARPS, bool GATE, bool PHASE1, bool YPART>
 __global__ void __launch_bounds__(32 * WARPS)
     scan_kernel(const __grid_constant__ ScanParams p)
 {
-    using Lay = Layout<io_t, NS, WARPS, GATE, PHASE1>;
+    // Scans that write per-direction partial outputs (several directions, short sequences,
+    // column-order boxes) keep one more tile in flight; the others keep the ring smaller so
+    // that more CTAs fit on an SM (both measured on B200).
+    constexpr int kStages = YPART ? 5 : 4;
+    using Lay = Layout<io_t, NS, WARPS, GATE, PHASE1, kStages>;
+    // the producer refills the stage released two tiles back and prepares the next tile, so at
+    // least four stages are needed for a tile to be in flight while the current one is scanned
+    static_assert(kStages >= 4, "the pipeline needs at least four stages");
     // fp32 inputs take the precise arithmetic, bf16 inputs the fast one
     constexpr bool PRECISE = sizeof(io_t) == 4;
     constexpr int DC = Lay::DC;
@@ -367,7 +385,6 @@ __global__ void __launch_bounds__(32 * WARPS)
     // Fill the stage of time tile `it` (warp 0).
     auto issue = [&](int64_t it) {
         const int st = static_cast<int>(it % kStages);
-        unsigned char* sb = smem + st * Lay::STAGE;
         const int64_t t0 = t_begin + it * kTile;
         const int rows = tile_rows(it);
         uint32_t bbytes, cbytes = 0;
@@ -383,15 +400,15 @@ __global__ void __launch_bounds__(32 * WARPS)
             else
                 tx += kUZ * static_cast<uint32_t>(rows) * row_bytes;
             mbar_expect_tx(&full[st], tx);
-            tma_2d(sb + Lay::OFF_DL, &p.tm_dl, static_cast<int32_t>(d0),
+            tma_2d(smem + Lay::OFF_DL + st * Lay::ROWS, &p.tm_dl, static_cast<int32_t>(d0),
                    static_cast<int32_t>(kb * p.L + t0), &full[st]);
             if (umode == 0) {
                 // reverse order: the box ends at the row of step t0
                 const int64_t prow = b * p.L + (dir == SS_DIR_FWD ? t0 : p.L - t0 - kTile);
-                tma_2d(sb + Lay::OFF_U, &p.tm_u, static_cast<int32_t>(d0),
+                tma_2d(smem + Lay::OFF_U + st * Lay::ROWS, &p.tm_u, static_cast<int32_t>(d0),
                        static_cast<int32_t>(prow), &full[st]);
                 if (Lay::HAS_Z)
-                    tma_2d(sb + Lay::OFF_Z, &p.tm_z, static_cast<int32_t>(d0),
+                    tma_2d(smem + Lay::OFF_Z + st * Lay::ROWS, &p.tm_z, static_cast<int32_t>(d0),
                            static_cast<int32_t>(prow), &full[st]);
             } else if (umode == 1) {
                 for (int sub = 0; sub < rows / 8; ++sub) {
@@ -399,29 +416,29 @@ __global__ void __launch_bounds__(32 * WARPS)
                     // column-major index of the lowest image row of the box
                     const int64_t c = dir == SS_DIR_COL ? tt : (p.L - 8 - tt);
                     const int64_t j = c / p.H, i = c - (c / p.H) * p.H;
-                    tma_3d(sb + Lay::OFF_U + 8 * sub * Lay::ROW, &p.tm_u3,
+                    tma_3d(smem + Lay::OFF_U + st * Lay::ROWS + 8 * sub * Lay::ROW, &p.tm_u3,
                            static_cast<int32_t>(d0), static_cast<int32_t>(j),
                            static_cast<int32_t>(b * p.H + i), &full[st]);
                     if (Lay::HAS_Z)
-                        tma_3d(sb + Lay::OFF_Z + 8 * sub * Lay::ROW, &p.tm_z3,
+                        tma_3d(smem + Lay::OFF_Z + st * Lay::ROWS + 8 * sub * Lay::ROW, &p.tm_z3,
                                static_cast<int32_t>(d0), static_cast<int32_t>(j),
                                static_cast<int32_t>(b * p.H + i), &full[st]);
                 }
             }
-            bulk_g2s(sb + Lay::OFF_BR, bsrc, bbytes, &full[st]);
+            bulk_g2s(smem + Lay::OFF_BR + st * Lay::BCRAW, bsrc, bbytes, &full[st]);
             if (Lay::HAS_C)
-                bulk_g2s(sb + Lay::OFF_CR, csrc, cbytes, &full[st]);
+                bulk_g2s(smem + Lay::OFF_CR + st * Lay::BCRAW, csrc, cbytes, &full[st]);
         }
         __syncwarp();
-        int64_t* orow = reinterpret_cast<int64_t*>(sb + Lay::OFF_OUT);
+        int64_t* orow = reinterpret_cast<int64_t*>(smem + Lay::OFF_OUT + st * Lay::OUT_STRIDE);
         for (int r = lane; r < rows; r += 32) {
             const int64_t pp = position(dir, p.L, p.H, p.W, t0 + r);
             orow[r] = (out_row0 + pp) * p.D + d0;
             if (umode == 2) {
-                bulk_g2s(sb + Lay::OFF_U + r * Lay::ROW, gu + (b * p.L + pp) * p.D + d0,
+                bulk_g2s(smem + Lay::OFF_U + st * Lay::ROWS + r * Lay::ROW, gu + (b * p.L + pp) * p.D + d0,
                          row_bytes, &full[st]);
                 if (Lay::HAS_Z)
-                    bulk_g2s(sb + Lay::OFF_Z + r * Lay::ROW, gz + (b * p.L + pp) * p.D + d0,
+                    bulk_g2s(smem + Lay::OFF_Z + st * Lay::ROWS + r * Lay::ROW, gz + (b * p.L + pp) * p.D + d0,
                              row_bytes, &full[st]);
             }
         }
@@ -434,7 +451,6 @@ __global__ void __launch_bounds__(32 * WARPS)
     // w = Delta*u / ln 2.
     auto convert = [&](int64_t it) {
         const int st = static_cast<int>(it % kStages);
-        unsigned char* sb = smem + st * Lay::STAGE;
         const int64_t t0 = t_begin + it * kTile;
         const int rows = tile_rows(it);
         uint32_t bytes;
@@ -442,9 +458,9 @@ __global__ void __launch_bounds__(32 * WARPS)
         bc_src(gB, t0, rows, bytes, bskip);
         if (Lay::HAS_C)
             bc_src(gC, t0, rows, bytes, cskip);
-        const io_t* br = reinterpret_cast<const io_t*>(sb + Lay::OFF_BR) + bskip;
-        const io_t* cr = reinterpret_cast<const io_t*>(sb + Lay::OFF_CR) + cskip;
-        float* bf = reinterpret_cast<float*>(sb + Lay::OFF_BF);
+        const io_t* br = reinterpret_cast<const io_t*>(smem + Lay::OFF_BR + st * Lay::BCRAW) + bskip;
+        const io_t* cr = reinterpret_cast<const io_t*>(smem + Lay::OFF_CR + st * Lay::BCRAW) + cskip;
+        float* bf = reinterpret_cast<float*>(smem + Lay::OFF_BF + st * Lay::BF_STRIDE);
         const float bscale = PRECISE ? 1.f : kLn2;
         if (!PRECISE && NS == 16 && p.N == 16 && bskip == 0 && cskip == 0) {
             // 16 bf16 rows of 16 values per tensor: lane l converts 8 values (16 bytes) of B and
@@ -547,7 +563,6 @@ __global__ void __launch_bounds__(32 * WARPS)
     for (int64_t it = 0; it < ntile_t && !failed; ++it) {
         const int st = static_cast<int>(it % kStages);
         const uint32_t ph = static_cast<uint32_t>((it / kStages) & 1);
-        unsigned char* sb = smem + st * Lay::STAGE;
         const int rows = tile_rows(it);
         if (*s_abort) {
             failed = true;
@@ -591,11 +606,11 @@ __global__ void __launch_bounds__(32 * WARPS)
         }
 
         if (active) {
-            const io_t* su = reinterpret_cast<const io_t*>(sb + Lay::OFF_U);
-            const io_t* sdl = reinterpret_cast<const io_t*>(sb + Lay::OFF_DL);
-            const io_t* sz = reinterpret_cast<const io_t*>(sb + Lay::OFF_Z);
-            const int64_t* orow = reinterpret_cast<const int64_t*>(sb + Lay::OFF_OUT);
-            const float* bf = reinterpret_cast<const float*>(sb + Lay::OFF_BF);
+            const io_t* su = reinterpret_cast<const io_t*>(smem + Lay::OFF_U + st * Lay::ROWS);
+            const io_t* sdl = reinterpret_cast<const io_t*>(smem + Lay::OFF_DL + st * Lay::ROWS);
+            const io_t* sz = reinterpret_cast<const io_t*>(smem + Lay::OFF_Z + st * Lay::ROWS);
+            const int64_t* orow = reinterpret_cast<const int64_t*>(smem + Lay::OFF_OUT + st * Lay::OUT_STRIDE);
+            const float* bf = reinterpret_cast<const float*>(smem + Lay::OFF_BF + st * Lay::BF_STRIDE);
             const float4* B4 = reinterpret_cast<const float4*>(bf);
             const float4* C4 = reinterpret_cast<const float4*>(bf + kTile * NS);
             if (PRECISE) {
@@ -673,8 +688,9 @@ __global__ void __launch_bounds__(32 * WARPS)
                         s_du[g] = dskip * uv;
                         s_g[g] = 1.f;
                         if (GATE) {
+                            // silu(z) = z * sigmoid(z), sigmoid(z) = (1 + tanh(z/2)) / 2
                             const float zv = Io<io_t>::ld(sz + (r ^ xmask) * DC + tid);
-                            s_g[g] = zv * rcp(1.f + ex2(-zv * kLog2e));
+                            s_g[g] = zv * fmaf(0.5f, tanh_approx(0.5f * zv), 0.5f);
                         }
                     }
 #pragma unroll
@@ -916,7 +932,7 @@ cudaError_t make_maps(ScanParams& p, bool need_z)
 template <typename io_t, int NS, bool GATE, bool PHASE1, bool YPART>
 cudaError_t launch_t(const ScanParams& p0, cudaStream_t stream)
 {
-    using Lay = Layout<io_t, NS, kWarps, GATE, PHASE1>;
+    using Lay = Layout<io_t, NS, kWarps, GATE, PHASE1, YPART ? 5 : 4>;
     auto kern = scan_kernel<io_t, NS, kWarps, GATE, PHASE1, YPART>;
     ScanParams p = p0;
     cudaError_t e = make_maps<io_t>(p, Lay::HAS_Z);
