@@ -18,7 +18,7 @@ Readings of the pages that the oracle fixes (each is listed with its reason in t
   * The gate is silu(z) = z*sigmoid(z) (Step 6, phi = SiLU); the Vim block's sigma(z) is read
     as the same gate.
   * With several directions every direction adds its own Dskip*u (each is a full S6 scan).
-  * The state starts at zero.
+  * The state starts at zero unless an initial state is given.
 """
 
 from __future__ import annotations
@@ -60,7 +60,7 @@ def _load():
             lib.ss_oracle_scan.restype = ctypes.c_int
             lib.ss_oracle_scan.argtypes = [i64, i64, i64, i64, i32, dp, i64, i64,
                                            dp, dp, dp, dp, dp, dp, dp, dp,
-                                           i32, i32, dp, dp, i32]
+                                           i32, i32, dp, dp, i32, dp]
             lib.ss_oracle_position.restype = ctypes.c_int64
             lib.ss_oracle_position.argtypes = [i32, i64, i64, i64, i64]
             lib.ss_oracle_max_threads.restype = ctypes.c_int
@@ -88,15 +88,17 @@ def _ptr(x):
 
 def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softplus=True,
                    dirs=(DIR_FORWARD,), H=0, W=0, zoh_exact=False, threads=None,
-                   return_last_state=True):
+                   return_last_state=True, initial_state=None):
     """Run the oracle.
 
     u, z: [batch, L, D]; delta: [K, batch, L, D]; B, C: [K, batch, L, N]; A: [D, N];
-    Dskip, delta_bias: [D] or None.  Inputs may be any real dtype; they are upcast to float64
-    exactly.  Returns (out [batch, L, D], last_state [K, batch, D, N]) in float64.
+    Dskip, delta_bias: [D] or None; initial_state: [K, batch, D, N] or None (zero).  Inputs
+    may be any real dtype; they are upcast to float64 exactly.  Returns (out [batch, L, D],
+    last_state [K, batch, D, N]) in float64.
     """
     u, delta, A, B, C = _f64(u), _f64(delta), _f64(A), _f64(B), _f64(C)
     Dskip, z, delta_bias = _f64(Dskip), _f64(z), _f64(delta_bias)
+    initial_state = _f64(initial_state)
     dirs_arr = np.ascontiguousarray(np.asarray(dirs, dtype=np.int32).reshape(-1))
     K = int(dirs_arr.size)
     if u.ndim != 3:
@@ -114,6 +116,8 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
     for v in (Dskip, delta_bias):
         if v is not None and v.shape != (D,):
             raise ValueError("Dskip and delta_bias must be [D]")
+    if initial_state is not None and initial_state.shape != (K, batch, D, N):
+        raise ValueError("initial_state must be [K, batch, D, N]")
     out = np.empty((batch, L, D), dtype=np.float64)
     last = np.empty((K, batch, D, N), dtype=np.float64) if return_last_state else None
     if threads is None:
@@ -121,7 +125,8 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
     rc = _load().ss_oracle_scan(batch, L, D, N, K, _ptr(dirs_arr), int(H), int(W),
                                 _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip),
                                 _ptr(z), _ptr(delta_bias), int(bool(softplus)),
-                                int(bool(zoh_exact)), _ptr(out), _ptr(last), int(threads))
+                                int(bool(zoh_exact)), _ptr(out), _ptr(last), int(threads),
+                                _ptr(initial_state))
     if rc != 0:
         raise ValueError("oracle rejected its arguments (code %d)" % rc)
     return out, last

@@ -9,7 +9,7 @@
  * What it computes, step by step, for every batch row b and channel d (all in double):
  *
  *   for each scan direction k (an ordering of the L positions):
- *     h[n] = 0 for all n                                  (no initial state is given)
+ *     h[n] = initial_state[k,b,d,n], or 0 without one     (the state before step 0)
  *     for t = 0 .. L-1:
  *       p     = spatial position visited at step t         (the direction's index map)
  *       Delta = softplus(delta[k,b,t,d] + bias[d])         ("Understanding Mamba from zero",
@@ -46,6 +46,7 @@
  *   z                    NULL means no gate
  *   out                  [batch, L, D]
  *   last_state           [K, batch, D, N] or NULL
+ *   initial_state        [K, batch, D, N] or NULL (zero)
  *
  * Parity is pinned by tests/test_oracle_pins.py against the LTI convolution form (eq. 3),
  * Theorem 1, the unrolled double sum, the Delta -> 0 limit, reversal and explicitly permuted
@@ -101,7 +102,8 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                    const double* B, const double* C, const double* Dskip,
                    const double* z, const double* delta_bias,
                    int32_t softplus, int32_t zoh_exact,
-                   double* out, double* last_state, int32_t nthreads)
+                   double* out, double* last_state, int32_t nthreads,
+                   const double* initial_state)
 {
     int bad = 0;
     if (batch < 0 || L < 0 || D < 0 || N < 1 || K < 1 || K > 4)
@@ -116,8 +118,13 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
             return ORACLE_BAD_ARG;
     }
     if (batch == 0 || L == 0 || D == 0) {
-        if (last_state)
-            memset(last_state, 0, sizeof(double) * (size_t)(K * batch * D * N));
+        /* no step is taken: the final state is the initial one */
+        if (last_state) {
+            if (initial_state)
+                memcpy(last_state, initial_state, sizeof(double) * (size_t)(K * batch * D * N));
+            else
+                memset(last_state, 0, sizeof(double) * (size_t)(K * batch * D * N));
+        }
         return ORACLE_OK;
     }
     if (nthreads <= 0)
@@ -136,7 +143,9 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                 memset(yacc, 0, sizeof(double) * (size_t)L);
                 for (int32_t k = 0; k < K; ++k) {
                     for (int64_t n = 0; n < N; ++n)
-                        h[n] = 0.0;
+                        h[n] = initial_state
+                                   ? initial_state[(((int64_t)k * batch + b) * D + d) * N + n]
+                                   : 0.0;
                     for (int64_t t = 0; t < L; ++t) {
                         const int64_t p = ss_oracle_position(dirs[k], L, H, W, t);
                         const double ut = u[(b * L + p) * D + d];

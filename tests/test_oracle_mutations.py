@@ -36,8 +36,11 @@ MUTATIONS = [
     ("last_state layout transposed", "last_state[(((int64_t)k * batch + b) * D + d) * N + n]",
      "last_state[(((int64_t)k * batch + b) * N + n) * D + d]"),
     ("state not reset between directions", "for (int64_t n = 0; n < N; ++n)\n"
-     "                        h[n] = 0.0;", "if (k == 0) for (int64_t n = 0; n < N; ++n)\n"
-     "                        h[n] = 0.0;"),
+     "                        h[n] = initial_state", "if (k == 0) for (int64_t n = 0; n < N; ++n)\n"
+     "                        h[n] = initial_state"),
+    ("initial state of the wrong direction", "initial_state[(((int64_t)k * batch + b) * D + d) * N + n]",
+     "initial_state[(((int64_t)0 * batch + b) * D + d) * N + n]"),
+    ("initial state ignored", "h[n] = initial_state\n", "h[n] = 0 && initial_state\n"),
 ]
 
 

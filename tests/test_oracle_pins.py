@@ -367,3 +367,62 @@ def test_golden_regression_fixture():
     assert rel_err(last, np.array(g["last_state"])) < 1e-13
     # the stored inputs' checksum guards the seeded generator as well
     assert abs(float(np.sum(f64["u"])) - g["sum_u"]) < 1e-9
+
+
+# ----------------------------------------------------------------------------- initial state
+
+@pytest.mark.parametrize("zoh", [False, True])
+def test_P6_initial_state_unrolled(zoh):
+    # with h_0 given: y_t gains sum_n C_t[n] exp(A_n sum_{r<=t} Delta_r) h_0[n], and the end state
+    # gains exp(A_n sum Delta) h_0[n]; the input terms are the unrolled double sum of P6
+    rng = np.random.default_rng(13)
+    batch, L, D, N, K = 2, 19, 3, 4, 2
+    c = rand_case(rng, batch, L, D, N, K=K)
+    h0 = rng.standard_normal((K, batch, D, N))
+    out, last = oracle.selective_scan(c["u"], c["delta"], c["A"], c["B"], c["C"], Dskip=c["Dskip"],
+                                      z=None, delta_bias=c["delta_bias"], softplus=True,
+                                      dirs=(FWD, REV), zoh_exact=zoh, initial_state=h0)
+    ref = np.zeros((batch, L, D))
+    href = np.zeros((K, batch, D, N))
+    for k in range(K):
+        order = np.arange(L) if k == 0 else np.arange(L)[::-1]
+        for b in range(batch):
+            for d in range(D):
+                dl = np_softplus(c["delta"][k, b, :, d] + c["delta_bias"][d])
+                cum = np.concatenate([[0.0], np.cumsum(dl)])
+                a = c["A"][d]
+                for t in range(L):
+                    decay0 = np.exp(a * cum[t + 1])
+                    acc = np.sum(c["C"][k, b, t] * decay0 * h0[k, b, d])
+                    for s in range(t + 1):
+                        bbar = (np.expm1(dl[s] * a) / a) if zoh else dl[s]
+                        acc += np.sum(c["C"][k, b, t] * np.exp(a * (cum[t + 1] - cum[s + 1])) *
+                                      bbar * c["B"][k, b, s]) * c["u"][b, order[s], d]
+                    ref[b, order[t], d] += acc + c["Dskip"][d] * c["u"][b, order[t], d]
+                hh = np.exp(a * cum[L]) * h0[k, b, d]
+                for s in range(L):
+                    bbar = (np.expm1(dl[s] * a) / a) if zoh else dl[s]
+                    hh = hh + np.exp(a * (cum[L] - cum[s + 1])) * bbar * c["B"][k, b, s] \
+                        * c["u"][b, order[s], d]
+                href[k, b, d] = hh
+    assert rel_err(out, ref) < 1e-11
+    assert rel_err(last, href) < 1e-11
+
+
+def test_P7_initial_state_continues_a_split_scan():
+    rng = np.random.default_rng(14)
+    batch, L, D, N, T = 2, 30, 3, 5, 11
+    c = rand_case(rng, batch, L, D, N)
+    args = dict(Dskip=c["Dskip"], delta_bias=c["delta_bias"], softplus=True)
+    out, last = oracle.selective_scan(c["u"], c["delta"], c["A"], c["B"], c["C"], z=c["z"], **args)
+    _, h1 = oracle.selective_scan(c["u"][:, :T], c["delta"][:, :, :T], c["A"], c["B"][:, :, :T],
+                                  c["C"][:, :, :T], z=c["z"][:, :T], **args)
+    out2, last2 = oracle.selective_scan(c["u"][:, T:], c["delta"][:, :, T:], c["A"],
+                                        c["B"][:, :, T:], c["C"][:, :, T:], z=c["z"][:, T:],
+                                        initial_state=h1, **args)
+    assert rel_err(out2, out[:, T:]) < 1e-13
+    assert rel_err(last2, last) < 1e-13
+    e = np.zeros((batch, 0, D))
+    _, l0 = oracle.selective_scan(e, np.zeros((1, batch, 0, D)), c["A"], np.zeros((1, batch, 0, N)),
+                                  np.zeros((1, batch, 0, N)), initial_state=h1)
+    assert np.array_equal(l0, h1)
