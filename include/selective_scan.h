@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define SS_ABI_VERSION 1
+#define SS_ABI_VERSION 2
 #define SS_MAX_DSTATE 16
 #define SS_MAX_DIRS 4
 
@@ -90,17 +90,23 @@ typedef struct {
     int32_t H, W;                /* image size; H*W == seqlen when a column order is used  */
 } ss_direction_map;
 
-/* Launch options for tuning, tests and timing; NULL or all-zero means "choose automatically". */
+/* Options and optional inputs; NULL or all-zero means "defaults, choose automatically". */
 typedef struct {
     int32_t segments;        /* split each sequence into this many segments (0 = auto)      */
     int32_t flags;           /* SS_FLAG_* bits                                               */
     void* scan_begin_event;  /* cudaEvent_t recorded on `stream` right before the main scan
                                 launch (the one that writes out), or NULL                    */
     void* scan_end_event;    /* cudaEvent_t recorded right after that launch, or NULL       */
-    int32_t reserved[4];     /* must be 0                                                    */
+    const float* initial_state; /* [K, batch, D, N] fp32 device array: the state h before
+                                   step 0 of each direction (eq. 2a's h_{-1}), or NULL for
+                                   zero; read only; must not overlap last_state             */
+    int32_t reserved[2];     /* must be 0                                                    */
 } ss_launch_opts;
 
 #define SS_FLAG_GENERIC_A 1 /* never use the exp-power shortcut for A[d,n] = (n+1)*A[d,0]   */
+#define SS_FLAG_ZOH_EXACT 2 /* Bbar = (exp(Delta*A) - 1) / A * B, eq. (4) exactly (A != 0;
+                               Delta*B where A == 0), instead of the first-order Delta*B;
+                               computed with the precise arithmetic for any io type        */
 
 /* Bytes of workspace that selective_scan_fwd needs for this problem and these options
  * (0 when it needs none).  Writes *bytes; validates shape, direction map and options the same

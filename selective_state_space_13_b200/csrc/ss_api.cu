@@ -31,6 +31,7 @@ struct Plan {
     int64_t seg_len;
     int flags;
     cudaEvent_t ev_begin, ev_end;
+    const float* init_state;
     // workspace layout (byte offsets, 0 size = unused)
     size_t off_carry_h, off_carry_s, off_ypart, bytes;
 };
@@ -98,14 +99,16 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
     int seg = 0;
     pl->flags = 0;
     pl->ev_begin = pl->ev_end = nullptr;
+    pl->init_state = nullptr;
     if (opts) {
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 2; ++i)
             if (opts->reserved[i] != 0)
                 return SS_ERR_UNSUPPORTED;
         if (opts->segments < 0 || opts->segments > kMaxSegments)
             return SS_ERR_UNSUPPORTED;
-        if (opts->flags & ~SS_FLAG_GENERIC_A)
+        if (opts->flags & ~(SS_FLAG_GENERIC_A | SS_FLAG_ZOH_EXACT))
             return SS_ERR_UNSUPPORTED;
+        pl->init_state = opts->initial_state;
         seg = opts->segments;
         pl->flags = opts->flags;
         pl->ev_begin = static_cast<cudaEvent_t>(opts->scan_begin_event);
@@ -199,7 +202,8 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
         if (p && !aligned(p, 16))
             return SS_ERR_ALIGN;
     for (const void* p : {static_cast<const void*>(A), static_cast<const void*>(Dskip),
-                          static_cast<const void*>(delta_bias), static_cast<const void*>(last_state)})
+                          static_cast<const void*>(delta_bias), static_cast<const void*>(last_state),
+                          static_cast<const void*>(pl.init_state)})
         if (p && !aligned(p, 4))
             return SS_ERR_ALIGN;
     if (pl.bytes > 0 && (!workspace || workspace_bytes < pl.bytes))
@@ -207,10 +211,14 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
 
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     if (!has_data) {
-        // no step is taken: the final state is the zero initial state
+        // no step is taken: the final state is the initial state (zero when none is given)
         if (last_state && has_state && pl.L == 0) {
             const size_t n = static_cast<size_t>(pl.K) * pl.batch * pl.D * pl.N * sizeof(float);
-            if (cudaMemsetAsync(last_state, 0, n, strm) != cudaSuccess)
+            const cudaError_t e =
+                pl.init_state
+                    ? cudaMemcpyAsync(last_state, pl.init_state, n, cudaMemcpyDeviceToDevice, strm)
+                    : cudaMemsetAsync(last_state, 0, n, strm);
+            if (e != cudaSuccess)
                 return SS_ERR_CUDA;
         }
         return SS_OK;
@@ -245,6 +253,8 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
     p.W = pl.W;
     p.softplus = softplus ? 1 : 0;
     p.force_generic = (pl.flags & SS_FLAG_GENERIC_A) ? 1 : 0;
+    p.zoh = (pl.flags & SS_FLAG_ZOH_EXACT) ? 1 : 0;
+    p.init_state = pl.init_state;
 
     if (pl.S > 1 && ss::launch_scan(p, pl.io, 1, strm) != cudaSuccess)
         return SS_ERR_CUDA;

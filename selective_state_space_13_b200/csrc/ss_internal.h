@@ -33,6 +33,7 @@ struct ScanParams {
     void* out;              // [batch, L, D] io (single direction) or null
     float* ypart;           // [K, batch, L, D] fp32 per-direction outputs (several directions)
     float* last_state;      // [K, batch, D, N] or null
+    const float* init_state;  // [K, batch, D, N] state before step 0, or null (zero)
     float* carry_h;         // [K, batch, S, D, N] end state of each segment scanned from zero
     float* carry_s;         // [K, batch, S, D] sum over the segment of Delta*log2(e)
     int64_t batch, L, D;
@@ -43,6 +44,7 @@ struct ScanParams {
     int32_t softplus;
     int32_t force_generic;  // 1: never take the A[d,n] = (n+1) A[d,0] shortcut
     int32_t col3d;          // 1: column orders load through tm_u3 / tm_z3 (H % 8 == 0)
+    int32_t zoh;            // 1: Bbar = (exp(Delta*A) - 1) / A * B (precise arithmetic)
 };
 
 struct MergeParams {

@@ -303,6 +303,8 @@ __global__ void __launch_bounds__(32 * WARPS)
     static_assert(kStages >= 4, "the pipeline needs at least four stages");
     // fp32 inputs take the precise arithmetic, bf16 inputs the fast one
     constexpr bool PRECISE = sizeof(io_t) == 4;
+    // the precise arithmetic also serves the exact-ZOH Bbar for any io type
+    const bool precise = PRECISE || p.zoh != 0;
     constexpr int DC = Lay::DC;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
@@ -461,8 +463,8 @@ __global__ void __launch_bounds__(32 * WARPS)
         const io_t* br = reinterpret_cast<const io_t*>(smem + Lay::OFF_BR + st * Lay::BCRAW) + bskip;
         const io_t* cr = reinterpret_cast<const io_t*>(smem + Lay::OFF_CR + st * Lay::BCRAW) + cskip;
         float* bf = reinterpret_cast<float*>(smem + Lay::OFF_BF + st * Lay::BF_STRIDE);
-        const float bscale = PRECISE ? 1.f : kLn2;
-        if (!PRECISE && NS == 16 && p.N == 16 && bskip == 0 && cskip == 0) {
+        const float bscale = precise ? 1.f : kLn2;
+        if (NS == 16 && p.N == 16 && sizeof(io_t) == 2 && bskip == 0 && cskip == 0) {
             // 16 bf16 rows of 16 values per tensor: lane l converts 8 values (16 bytes) of B and
             // 8 of C; rows past the tile's end become 0
             static_assert(kTile * 16 * 2 == 32 * 16, "one 16-byte chunk per lane and tensor");
@@ -524,6 +526,13 @@ __global__ void __launch_bounds__(32 * WARPS)
 #pragma unroll
     for (int j = 0; j < NS / 2; ++j)
         kst2[j] = make_float2(0.f, 0.f);
+    if (!PHASE1 && active && p.init_state) {
+        const float* h0 = p.init_state + (kb * p.D + d) * p.N;
+#pragma unroll
+        for (int n = 0; n < NS; ++n)
+            if (n < p.N)
+                kst[n] = h0[n];
+    }
     if (!PHASE1 && seg > 0 && active) {
         // fold the carries of segments 0..seg-1: h <- exp(A * sumDelta_s) * h + h_s
         for (int s = 0; s < seg; ++s) {
@@ -613,9 +622,10 @@ __global__ void __launch_bounds__(32 * WARPS)
             const float* bf = reinterpret_cast<const float*>(smem + Lay::OFF_BF + st * Lay::BF_STRIDE);
             const float4* B4 = reinterpret_cast<const float4*>(bf);
             const float4* C4 = reinterpret_cast<const float4*>(bf + kTile * NS);
-            if (PRECISE) {
-                // h = (1 + expm1(Delta*A)) h + Delta*u*B without rounding Abar to fp32, so the
-                // per-step error does not grow with the memory length 1/|Delta*A|
+            if (precise) {
+                // h = (1 + expm1(Delta*A)) h + Bbar*u*B without rounding Abar to fp32, so the
+                // per-step error does not grow with the memory length 1/|Delta*A|; Bbar is Delta,
+                // or expm1(Delta*A)/A with the exact ZOH
                 for (int r = 0; r < rows; ++r) {
                     const float uv = Io<io_t>::ld(su + (r ^ xmask) * DC + tid);
                     const float dr = Io<io_t>::ld(sdl + r * DC + tid);
@@ -639,7 +649,8 @@ __global__ void __launch_bounds__(32 * WARPS)
                         for (int j = 0; j < 4; ++j) {
                             const int n = n4 * 4 + j;
                             const float em1 = expm1_acc(dt * a_l[n]);
-                            kst[n] = fmaf(em1, kst[n], fmaf(w, bv[j], kst[n]));
+                            const float wb = p.zoh && a_l[n] != 0.f ? (em1 / a_l[n]) * uv : w;
+                            kst[n] = fmaf(em1, kst[n], fmaf(wb, bv[j], kst[n]));
                             if (!PHASE1)
                                 yp = fmaf(cv[j], kst[n], yp);
                         }

@@ -23,6 +23,7 @@ SS_ERR_SCRATCH_LIMIT = 10
 SS_F32, SS_BF16 = 0, 1
 SS_DIR_FWD, SS_DIR_REV, SS_DIR_COL, SS_DIR_COL_REV = 0, 1, 2, 3
 SS_FLAG_GENERIC_A = 1
+SS_FLAG_ZOH_EXACT = 2
 SS_MAX_DSTATE = 16
 SS_MAX_DIRS = 4
 
@@ -50,7 +51,7 @@ class SsDirectionMap(ctypes.Structure):
 class SsLaunchOpts(ctypes.Structure):
     _fields_ = [("segments", ctypes.c_int32), ("flags", ctypes.c_int32),
                 ("scan_begin_event", ctypes.c_void_p), ("scan_end_event", ctypes.c_void_p),
-                ("reserved", ctypes.c_int32 * 4)]
+                ("initial_state", ctypes.c_void_p), ("reserved", ctypes.c_int32 * 2)]
 
 
 class ScanError(RuntimeError):
@@ -151,12 +152,14 @@ def make_dirmap(dirs=(SS_DIR_FWD,), H=0, W=0) -> SsDirectionMap:
     return m
 
 
-def make_opts(segments=0, flags=0, events=None) -> SsLaunchOpts:
+def make_opts(segments=0, flags=0, events=None, initial_state=0) -> SsLaunchOpts:
     """events: optional (begin, end) torch.cuda.Event pair, recorded by the library around its
     main scan launch on the call's stream (each must have been recorded once before, so that
-    its CUDA event exists)."""
+    its CUDA event exists).  initial_state: device address of a [K, batch, D, N] fp32 array
+    (0 = zero state)."""
     o = SsLaunchOpts()
     o.segments, o.flags = int(segments), int(flags)
+    o.initial_state = int(initial_state) or None
     if events is not None:
         o.scan_begin_event = int(events[0].cuda_event) or None
         o.scan_end_event = int(events[1].cuda_event) or None
@@ -262,12 +265,14 @@ def _workspace(nbytes, device):
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                        dirs=(SS_DIR_FWD,), H=0, W=0, out=None, last_state=None,
                        return_last_state=False, workspace=None, stream=None, segments=0,
-                       flags=0, events=None):
+                       flags=0, events=None, initial_state=None, zoh_exact=False):
     """Selective scan forward on CUDA tensors.
 
     u, z: [batch, L, D]; delta: [K, batch, L, D] (or [batch, L, D] when K = 1); B, C:
     [K, batch, L, N] (or [batch, L, N]); A: [D, N] float32; D (skip) and delta_bias: [D] float32.
     u, delta, B, C, z share one dtype (float32 or bfloat16); out has that dtype.
+    initial_state: [K, batch, D, N] float32 state before step 0 (None = zero); zoh_exact: use
+    Bbar = (exp(Delta*A) - 1) / A * B instead of Delta*B.
     Returns out, or (out, last_state [K, batch, D, N] float32) with return_last_state.
     """
     import torch
@@ -299,9 +304,12 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     if return_last_state and last_state is None:
         last_state = torch.empty((K, batch, Dm, N), dtype=torch.float32, device=device)
     _check(last_state, "last_state", (K, batch, Dm, N), torch.float32, device)
+    _check(initial_state, "initial_state", (K, batch, Dm, N), torch.float32, device)
+    if zoh_exact:
+        flags = int(flags) | SS_FLAG_ZOH_EXACT
     shape = make_shape(batch, L, Dm, N, _io_code(io))
     dmap = make_dirmap(dirs, H, W)
-    opts = make_opts(segments, flags, events)
+    opts = make_opts(segments, flags, events, _ptr(initial_state))
     nws = selective_scan_workspace_size(shape, dmap, opts)
     if workspace is None and nws > 0:
         workspace = _workspace(nws, device)

@@ -52,20 +52,24 @@ def out_to_f64(t):
 
 
 def run_gpu(inp, dev_inputs=None, device="cuda:0", segments=0, flags=0, use_z=True, use_D=True,
-            use_bias=True, softplus=None):
+            use_bias=True, softplus=None, initial_state=None, zoh_exact=False):
+    import torch
     from selective_state_space_13_b200 import scan
     w = inp["workload"]
     t = dev_inputs if dev_inputs is not None else to_device(inp, device)
+    h0 = None if initial_state is None else \
+        torch.from_numpy(np.ascontiguousarray(initial_state, dtype=np.float32)).to(t["u"].device)
     out, last = scan.selective_scan_fwd(
         t["u"], t["delta"], t["A"], t["B"], t["C"], D=t["D"] if use_D else None,
         z=t["z"] if use_z else None, delta_bias=t["delta_bias"] if use_bias else None,
         softplus=w.softplus if softplus is None else softplus, dirs=w.dirs, H=w.H, W=w.W,
-        return_last_state=True, segments=segments, flags=flags)
+        return_last_state=True, segments=segments, flags=flags, initial_state=h0,
+        zoh_exact=zoh_exact)
     return out, last
 
 
 def run_oracle(inp, channels=None, batches=None, use_z=True, use_D=True, use_bias=True,
-               softplus=None):
+               softplus=None, initial_state=None, zoh_exact=False):
     w = inp["workload"]
     f = wl.inputs_f64(inp, channels=channels, batches=batches)
     return oracle.selective_scan(f["u"], f["delta"], f["A"], f["B"], f["C"],
@@ -73,4 +77,5 @@ def run_oracle(inp, channels=None, batches=None, use_z=True, use_D=True, use_bia
                                  z=f["z"] if use_z else None,
                                  delta_bias=f["delta_bias"] if use_bias else None,
                                  softplus=w.softplus if softplus is None else softplus,
-                                 dirs=w.dirs, H=w.H, W=w.W)
+                                 dirs=w.dirs, H=w.H, W=w.W, initial_state=initial_state,
+                                 zoh_exact=zoh_exact)

@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol():
     assert set(names) == set(scan.EXPORTED), names
     for name in names:
         assert hasattr(lib, name), name
-    assert scan.ss_abi_version() == 1
+    assert scan.ss_abi_version() == 2
 
 
 def test_status_strings():
@@ -109,7 +109,7 @@ def test_null_alignment_and_workspace_errors():
                                      FAKE, need - 1, 0)
     assert st == 8
     # unknown option bits / reserved fields
-    o = scan.make_opts(flags=2)
+    o = scan.make_opts(flags=4)
     with pytest.raises(scan.ScanError):
         scan.selective_scan_workspace_size(sh, None, o)
     o = scan.make_opts(segments=-1)

@@ -134,6 +134,41 @@ def test_repeat_calls_identical(cuda_device):
     assert bool((o1 == o2).all()) and bool((l1 == l2).all())
 
 
+@pytest.mark.parametrize("segments", [1, 3])
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F32])
+def test_initial_state(cuda_device, dtype, segments):
+    w = wl.variant("vim", name="h0", batch=2, seqlen=250, dim=64, dtype=dtype, seed=97)
+    inp = wl.make_inputs(w)
+    h0 = np.random.default_rng(8).standard_normal((w.K, w.batch, w.dim, w.dstate)).astype(np.float32)
+    _check(inp, cuda_device, segments=segments, initial_state=h0)
+
+
+@pytest.mark.parametrize("case", ["bf16", "f32", "bf16_split", "f32_genericA"])
+def test_exact_zoh(cuda_device, case):
+    dtype = wl.F32 if case.startswith("f32") else wl.BF16
+    w = wl.variant("m130", name="zoh", batch=2, seqlen=180, dim=72, dtype=dtype, seed=98)
+    inp = wl.make_inputs(w)
+    if case == "f32_genericA":
+        rng = np.random.default_rng(9)
+        inp["A"] = (-rng.uniform(0.05, 3.0, size=inp["A"].shape)).astype(np.float32)
+        inp["A"][3, 5] = 0.0  # A = 0: Bbar falls back to Delta*B
+    segments = 3 if case == "bf16_split" else 1
+    _check(inp, cuda_device, segments=segments, zoh_exact=True)
+
+
+def test_initial_state_with_empty_sequence(cuda_device):
+    import torch
+    from selective_state_space_13_b200 import scan
+    h0 = torch.randn((1, 2, 16, 4), device=cuda_device)
+    u = torch.empty((2, 0, 16), device=cuda_device)
+    e = torch.empty((1, 2, 0, 16), device=cuda_device)
+    bc = torch.empty((1, 2, 0, 4), device=cuda_device)
+    out, last = scan.selective_scan_fwd(u, e, -torch.ones((16, 4), device=cuda_device), bc, bc,
+                                        return_last_state=True, initial_state=h0)
+    torch.cuda.synchronize()
+    assert torch.equal(last, h0)
+
+
 def test_device_status_clean(cuda_device):
     from selective_state_space_13_b200 import scan
     assert scan.selective_scan_device_status(clear=True) == scan.SS_OK
