@@ -38,6 +38,9 @@ UNIT = "GB/s"
 DEFAULT_WORKLOAD = "m130"
 FALLBACK_HBM_GBS = 6650.0
 FLUSH_BYTES = 256 << 20
+# FP32 work of one state update in the form the kernels compute (the exp(Delta*A) of a state
+# taken as one multiply of the power chain, the state multiply-add, the readout multiply-add)
+FLOP_PER_UPDATE = 5
 # workloads whose description states that last_state is returned
 RETURNS_LAST_STATE = {"tiny", "long"}
 
@@ -319,6 +322,12 @@ def run_ours(args):
     updates_s = world * w.updates() / (step_ms * 1e-3)
     peak, peak_src, peaks = load_peaks()
     achieved = nbytes / (kern_ms * 1e-3) / 1e9
+    # ALU roofline: FP32 FLOPs the method needs per state update, over the FP32 peak derived
+    # from B200's unit counts and the clock (148 SMs x 128 FP32 lanes x 2 FLOP per FMA)
+    sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+    fp32_peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    flops = FLOP_PER_UPDATE * w.updates()
+    alu_achieved = flops / (kern_ms * 1e-3) / 1e12
 
     # ---- end to end: pinned host inputs -> device, scan, out -> pinned host, every step
     e2e = None
@@ -389,12 +398,17 @@ def run_ours(args):
                    "segments": args.segments or "auto", "workspace_bytes": ws_bytes},
         "hbm_frac_of_peak": value / world / peak,
         "updates_per_s": updates_s,
-        "roofline": {"bound": "hbm", "kernel": "scan_kernel (main scan launch)",
-                     "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": peak_src,
-                     "algorithmic_bytes_per_launch": nbytes,
-                     "kernel_ms": kern_ms},
+        "roofline": {"bound": "alu", "kernel": "scan_kernel (main scan launch)",
+                     "achieved": alu_achieved, "peak": fp32_peak, "unit": "TFLOP/s",
+                     "frac": alu_achieved / fp32_peak, "traffic": traffic,
+                     "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x %.0f MHz "
+                                    "(no measured FP32 figure in MEASURED_PEAKS.json)" % sm_mhz,
+                     "algorithmic_flop_per_launch": flops,
+                     "flop_per_update": FLOP_PER_UPDATE,
+                     "kernel_ms": kern_ms,
+                     "hbm": {"achieved": achieved, "peak": peak, "unit": "GB/s",
+                             "frac": achieved / peak, "peak_source": peak_src,
+                             "algorithmic_bytes_per_launch": nbytes}},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": sampler.report(),
         "e2e": e2e,

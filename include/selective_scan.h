@@ -107,6 +107,11 @@ typedef struct {
 #define SS_FLAG_ZOH_EXACT 2 /* Bbar = (exp(Delta*A) - 1) / A * B, eq. (4) exactly (A != 0;
                                Delta*B where A == 0), instead of the first-order Delta*B;
                                computed with the precise arithmetic for any io type        */
+#define SS_FLAG_TEST_WAIT_TIMEOUT 8 /* test hook for failure detection: every CTA waits (20 ms
+                                       at most) on a barrier that nothing completes, gives up,
+                                       records SS_ERR_DEVICE_TIMEOUT for
+                                       selective_scan_device_status and returns without
+                                       touching its outputs                                 */
 
 /* Bytes of workspace that selective_scan_fwd needs for this problem and these options
  * (0 when it needs none).  Writes *bytes; validates shape, direction map and options the same

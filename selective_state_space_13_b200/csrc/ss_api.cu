@@ -106,7 +106,7 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
                 return SS_ERR_UNSUPPORTED;
         if (opts->segments < 0 || opts->segments > kMaxSegments)
             return SS_ERR_UNSUPPORTED;
-        if (opts->flags & ~(SS_FLAG_GENERIC_A | SS_FLAG_ZOH_EXACT))
+        if (opts->flags & ~(SS_FLAG_GENERIC_A | SS_FLAG_ZOH_EXACT | SS_FLAG_TEST_WAIT_TIMEOUT))
             return SS_ERR_UNSUPPORTED;
         pl->init_state = opts->initial_state;
         seg = opts->segments;
@@ -254,6 +254,7 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
     p.softplus = softplus ? 1 : 0;
     p.force_generic = (pl.flags & SS_FLAG_GENERIC_A) ? 1 : 0;
     p.zoh = (pl.flags & SS_FLAG_ZOH_EXACT) ? 1 : 0;
+    p.test_timeout = (pl.flags & SS_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
     p.init_state = pl.init_state;
 
     if (pl.S > 1 && ss::launch_scan(p, pl.io, 1, strm) != cudaSuccess)

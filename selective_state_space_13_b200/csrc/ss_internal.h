@@ -45,6 +45,7 @@ struct ScanParams {
     int32_t force_generic;  // 1: never take the A[d,n] = (n+1) A[d,0] shortcut
     int32_t col3d;          // 1: column orders load through tm_u3 / tm_z3 (H % 8 == 0)
     int32_t zoh;            // 1: Bbar = (exp(Delta*A) - 1) / A * B (precise arithmetic)
+    int32_t test_timeout;   // 1: test hook, wait on a barrier nothing completes and report
 };
 
 struct MergeParams {

@@ -24,6 +24,8 @@ SS_F32, SS_BF16 = 0, 1
 SS_DIR_FWD, SS_DIR_REV, SS_DIR_COL, SS_DIR_COL_REV = 0, 1, 2, 3
 SS_FLAG_GENERIC_A = 1
 SS_FLAG_ZOH_EXACT = 2
+SS_FLAG_TEST_WAIT_TIMEOUT = 8
+SS_ERR_DEVICE_TIMEOUT = 9
 SS_MAX_DSTATE = 16
 SS_MAX_DIRS = 4
 

@@ -169,6 +169,27 @@ def test_initial_state_with_empty_sequence(cuda_device):
     assert torch.equal(last, h0)
 
 
+def test_bounded_wait_gives_up_and_reports(cuda_device):
+    # a wait on a barrier that nothing completes must run out, leave the outputs alone, report
+    # SS_ERR_DEVICE_TIMEOUT, and leave the context usable
+    import torch
+    from selective_state_space_13_b200 import scan
+    w = wl.variant("m130", name="tmo", batch=1, seqlen=64, dim=64, seed=99)
+    inp = wl.make_inputs(w)
+    t = to_device(inp, cuda_device)
+    assert scan.selective_scan_device_status(clear=True) == scan.SS_OK
+    sentinel = torch.full_like(t["u"], 7.0)
+    out = scan.selective_scan_fwd(t["u"], t["delta"], t["A"], t["B"], t["C"], D=t["D"], z=t["z"],
+                                  delta_bias=t["delta_bias"], out=sentinel,
+                                  flags=scan.SS_FLAG_TEST_WAIT_TIMEOUT)
+    assert scan.selective_scan_device_status(clear=False) == scan.SS_ERR_DEVICE_TIMEOUT
+    assert torch.all(out == 7.0)
+    assert scan.selective_scan_device_status(clear=True) == scan.SS_ERR_DEVICE_TIMEOUT
+    assert scan.selective_scan_device_status(clear=True) == scan.SS_OK
+    _check(inp, cuda_device)
+    assert scan.selective_scan_device_status(clear=True) == scan.SS_OK
+
+
 def test_device_status_clean(cuda_device):
     from selective_state_space_13_b200 import scan
     assert scan.selective_scan_device_status(clear=True) == scan.SS_OK
