@@ -398,7 +398,9 @@ def run_ours(args):
                    "segments": args.segments or "auto", "workspace_bytes": ws_bytes},
         "hbm_frac_of_peak": value / world / peak,
         "updates_per_s": updates_s,
-        "roofline": {"bound": "alu", "kernel": "scan_kernel (main scan launch)",
+        "roofline": {"bound": "alu",
+                     "kernel": "scan pipeline: scan_kernel launches (segment aggregates, if any, "
+                               "and the scan; the direction merge excluded)",
                      "achieved": alu_achieved, "peak": fp32_peak, "unit": "TFLOP/s",
                      "frac": alu_achieved / fp32_peak, "traffic": traffic,
                      "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x %.0f MHz "

@@ -94,9 +94,11 @@ typedef struct {
 typedef struct {
     int32_t segments;        /* split each sequence into this many segments (0 = auto)      */
     int32_t flags;           /* SS_FLAG_* bits                                               */
-    void* scan_begin_event;  /* cudaEvent_t recorded on `stream` right before the main scan
-                                launch (the one that writes out), or NULL                    */
-    void* scan_end_event;    /* cudaEvent_t recorded right after that launch, or NULL       */
+    void* scan_begin_event;  /* cudaEvent_t recorded on `stream` right before the scan
+                                pipeline (the segment-aggregate launch, if any, and the scan
+                                launch that writes out or the per-direction partials), or NULL */
+    void* scan_end_event;    /* cudaEvent_t recorded right after that pipeline (before the
+                                direction merge), or NULL                                    */
     const float* initial_state; /* [K, batch, D, N] fp32 device array: the state h before
                                    step 0 of each direction (eq. 2a's h_{-1}), or NULL for
                                    zero; read only; must not overlap last_state             */

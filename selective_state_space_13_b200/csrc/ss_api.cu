@@ -257,9 +257,11 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
     p.test_timeout = (pl.flags & SS_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
     p.init_state = pl.init_state;
 
-    if (pl.S > 1 && ss::launch_scan(p, pl.io, 1, strm) != cudaSuccess)
-        return SS_ERR_CUDA;
+    // the timing events bracket the scan pipeline: the segment-aggregate launch (if any) and
+    // the scan launch, which may overlap (nothing is recorded between them)
     if (pl.ev_begin && cudaEventRecord(pl.ev_begin, strm) != cudaSuccess)
+        return SS_ERR_CUDA;
+    if (pl.S > 1 && ss::launch_scan(p, pl.io, 1, strm) != cudaSuccess)
         return SS_ERR_CUDA;
     if (ss::launch_scan(p, pl.io, 0, strm) != cudaSuccess)
         return SS_ERR_CUDA;

@@ -154,6 +154,18 @@ __device__ __forceinline__ void tma_3d(void* dst, const CUtensorMap* map, int32_
         : "memory");
 }
 
+// Programmatic dependent launch: let the next kernel in the stream start (launch_dependents);
+// wait until the previous kernel has finished and its writes are visible (wait).
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ float ex2(float x)
 {
     float y;
@@ -317,14 +329,16 @@ __global__ void __launch_bounds__(32 * WARPS)
     const int lane = tid & 31;
     const int warp = tid >> 5;
 
-    // ---- which (direction, batch row, segment, channel tile) this CTA owns
+    // ---- which (segment, direction, batch row, channel tile) this CTA owns; segments are the
+    // slowest index, so the first CTAs of a scan launch are the segment-0 ones, which need no
+    // carry and can run while the segment aggregates are still being computed
     const int64_t ntiles = (p.D + DC - 1) / DC;
-    const int nseg = PHASE1 ? (p.S - 1) : p.S;
+    const int64_t per_seg = ntiles * p.batch * p.K;
     int64_t blk = blockIdx.x;
+    const int seg = static_cast<int>(blk / per_seg);
+    blk -= static_cast<int64_t>(seg) * per_seg;
     const int64_t tile = blk % ntiles;
     blk /= ntiles;
-    const int seg = static_cast<int>(blk % nseg);
-    blk /= nseg;
     const int64_t b = blk % p.batch;
     const int k = static_cast<int>(blk / p.batch);
     // constant indices keep the parameter array out of local memory
@@ -357,6 +371,9 @@ __global__ void __launch_bounds__(32 * WARPS)
         fence_mbar_init();
     }
     __syncthreads();
+    // the next launch (the scan after the aggregates, the merge after the scan) may start now;
+    // it waits for this grid's results itself where it needs them
+    pdl_launch_dependents();
     if (p.test_timeout) {
         // failure-detection test hook: nobody arrives on ready[0], so this bounded wait gives
         // up; no copy has been issued yet, so the CTA can return at once
@@ -541,16 +558,20 @@ __global__ void __launch_bounds__(32 * WARPS)
             if (n < p.N)
                 kst[n] = h0[n];
     }
+    if (!PHASE1 && seg > 0) {
+        // the carries come from the aggregate launch just before this one
+        pdl_wait();
+    }
     if (!PHASE1 && seg > 0 && active) {
         // fold the carries of segments 0..seg-1: h <- exp(A * sumDelta_s) * h + h_s
         for (int s = 0; s < seg; ++s) {
             const int64_t ci = (kb * p.S + s) * p.D + d;
-            const float sd = p.carry_s[ci];
+            const float sd = __ldcg(p.carry_s + ci);
             const float* ch = p.carry_h + ci * p.N;
 #pragma unroll
             for (int n = 0; n < NS; ++n)
                 if (n < p.N)
-                    kst[n] = ex2(a_l[n] * sd) * kst[n] + ch[n];
+                    kst[n] = ex2(a_l[n] * sd) * kst[n] + __ldcg(ch + n);
         }
     }
     float dsum = 0.f;  // sum of Delta*log2(e) over this segment (aggregate launch)
@@ -857,6 +878,7 @@ __device__ __forceinline__ float silu_f(float z) { return z * rcp(1.f + ex2(-z *
 template <typename io_t, bool GATE, int K>
 __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ MergeParams p)
 {
+    pdl_wait();  // the per-direction outputs come from the scan launch just before
     const int64_t plane = p.rows * p.D;
     const int64_t n4 = plane / 4;  // D is a multiple of 4
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
@@ -887,6 +909,25 @@ __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ Merg
 // ---------------------------------------------------------------------------- dispatch
 
 constexpr int kWarps = 2;
+
+// Launch `kern(p)`; with `dependent`, the launch may begin before the previous kernel in the
+// stream has finished (programmatic dependent launch).
+template <typename Kern, typename P>
+cudaError_t launch_ex(Kern kern, unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                      bool dependent, const P& p)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = dependent ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+}
 
 // cuTensorMapEncodeTiled, looked up once through the runtime (no link-time libcuda dependency).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
@@ -965,8 +1006,11 @@ cudaError_t launch_t(const ScanParams& p0, cudaStream_t stream)
     const int64_t nblocks = ntiles * nseg * p.batch * p.K;
     if (nblocks <= 0)
         return cudaSuccess;
-    kern<<<static_cast<unsigned int>(nblocks), 32 * kWarps, Lay::BYTES, stream>>>(p);
-    return cudaGetLastError();
+    // a scan launch that follows the aggregate launch may start before it ends (its segment-0
+    // CTAs need nothing from it; the others wait for it in the kernel)
+    const bool after_aggregates = !PHASE1 && p.S > 1;
+    return launch_ex(kern, static_cast<unsigned>(nblocks), 32 * kWarps, Lay::BYTES, stream,
+                     after_aggregates, p);
 }
 
 template <typename io_t, int NS>
@@ -1001,12 +1045,13 @@ cudaError_t launch_scan(const ScanParams& p, int io_dtype, int phase1, cudaStrea
 }
 
 template <typename io_t, bool GATE>
-void merge_k(const MergeParams& p, unsigned blocks, cudaStream_t stream)
+cudaError_t merge_k(const MergeParams& p, unsigned blocks, cudaStream_t stream)
 {
+    // the merge may launch before the scan ends; it waits for the scan's outputs itself
     switch (p.K) {
-    case 2: merge_kernel<io_t, GATE, 2><<<blocks, 256, 0, stream>>>(p); break;
-    case 3: merge_kernel<io_t, GATE, 3><<<blocks, 256, 0, stream>>>(p); break;
-    default: merge_kernel<io_t, GATE, 4><<<blocks, 256, 0, stream>>>(p); break;
+    case 2: return launch_ex(merge_kernel<io_t, GATE, 2>, blocks, 256, 0, stream, true, p);
+    case 3: return launch_ex(merge_kernel<io_t, GATE, 3>, blocks, 256, 0, stream, true, p);
+    default: return launch_ex(merge_kernel<io_t, GATE, 4>, blocks, 256, 0, stream, true, p);
     }
 }
 
@@ -1024,10 +1069,9 @@ cudaError_t launch_merge(const MergeParams& p, int io_dtype, cudaStream_t stream
     const unsigned nb = static_cast<unsigned>(blocks);
     const bool gate = p.z != nullptr;
     if (io_dtype == SS_BF16)
-        gate ? merge_k<__nv_bfloat16, true>(p, nb, stream) : merge_k<__nv_bfloat16, false>(p, nb, stream);
-    else
-        gate ? merge_k<float, true>(p, nb, stream) : merge_k<float, false>(p, nb, stream);
-    return cudaGetLastError();
+        return gate ? merge_k<__nv_bfloat16, true>(p, nb, stream)
+                    : merge_k<__nv_bfloat16, false>(p, nb, stream);
+    return gate ? merge_k<float, true>(p, nb, stream) : merge_k<float, false>(p, nb, stream);
 }
 
 int64_t position_host(int32_t dir, int64_t L, int32_t H, int32_t W, int64_t t)
