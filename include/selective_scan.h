@@ -77,7 +77,7 @@ typedef enum { SS_DIR_FWD = 0, SS_DIR_REV = 1, SS_DIR_COL = 2, SS_DIR_COL_REV = 
 
 typedef struct {
     int64_t batch;    /* b  >= 0                                                   */
-    int64_t seqlen;   /* L  >= 0, < 2^31                                           */
+    int64_t seqlen;   /* L  >= 0; batch*L*4 < 2^31 and L*dim < 2^31               */
     int64_t dim;      /* D  >= 0 channels                                          */
     int64_t dstate;   /* N  in 1..SS_MAX_DSTATE                                    */
     int32_t io_dtype; /* ss_dtype of u, delta, z, B, C and out                     */

@@ -57,8 +57,9 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
         return SS_ERR_UNSUPPORTED;
     if (s->batch > (int64_t{1} << 24) || s->dim > (int64_t{1} << 24))
         return SS_ERR_SHAPE;
-    // tile coordinates are 32-bit: every direction's rows must be addressable
-    if (s->batch * s->seqlen * SS_MAX_DIRS > kMaxSeqlen)
+    // tile coordinates are 32-bit: every direction's rows must be addressable; a position's
+    // element offset inside one sequence (L * D) must fit in 32 bits as well
+    if (s->batch * s->seqlen * SS_MAX_DIRS > kMaxSeqlen || s->seqlen * s->dim > kMaxSeqlen)
         return SS_ERR_SHAPE;
     const int esz = s->io_dtype == SS_BF16 ? 2 : 4;
     if ((s->dim * esz) % 16 != 0)

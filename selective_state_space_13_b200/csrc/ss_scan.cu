@@ -283,8 +283,8 @@ struct Layout {
     static constexpr int OFF_BF = OFF_CR + (HAS_C ? STAGES * BCRAW : 0);  // fp32 B, then fp32 C
     static constexpr int BF_ONE = kTile * NS * 4;
     static constexpr int BF_STRIDE = BF_ONE * (HAS_C ? 2 : 1);
-    static constexpr int OFF_OUT = OFF_BF + STAGES * BF_STRIDE;           // int64 row offsets
-    static constexpr int OUT_STRIDE = kTile * 8;
+    static constexpr int OFF_OUT = OFF_BF + STAGES * BF_STRIDE;           // int32 row offsets
+    static constexpr int OUT_STRIDE = kTile * 4;
     static constexpr int OFF_BAR = OFF_OUT + STAGES * OUT_STRIDE;         // full, ready, empty
     static constexpr int OFF_FLAG = OFF_BAR + 3 * STAGES * 8;
     static constexpr int BYTES = OFF_FLAG + 16;
@@ -358,8 +358,9 @@ __global__ void __launch_bounds__(32 * WARPS)
     const io_t* gB = static_cast<const io_t*>(p.B);
     const io_t* gC = static_cast<const io_t*>(p.C);
     const int64_t kb = static_cast<int64_t>(k) * p.batch + b;  // (direction, batch) row block
-    // output rows: out[b, p, :] for one direction, ypart[k, b, p, :] for several
-    const int64_t out_row0 = p.ypart ? kb * p.L : b * p.L;
+    // output rows: out[b, p, :] for one direction, ypart[k, b, p, :] for several; a row's
+    // element offset from this CTA's base (row 0 of its block, channel d0) fits in 32 bits
+    const int64_t out_base = (p.ypart ? kb * p.L : b * p.L) * p.D + d0;
 
     if (tid == 0) {
         *s_abort = 0;
@@ -457,10 +458,10 @@ __global__ void __launch_bounds__(32 * WARPS)
                 bulk_g2s(smem + Lay::OFF_CR + st * Lay::BCRAW, csrc, cbytes, &full[st]);
         }
         __syncwarp();
-        int64_t* orow = reinterpret_cast<int64_t*>(smem + Lay::OFF_OUT + st * Lay::OUT_STRIDE);
+        int32_t* orow = reinterpret_cast<int32_t*>(smem + Lay::OFF_OUT + st * Lay::OUT_STRIDE);
         for (int r = lane; r < rows; r += 32) {
             const int64_t pp = position(dir, p.L, p.H, p.W, t0 + r);
-            orow[r] = (out_row0 + pp) * p.D + d0;
+            orow[r] = static_cast<int32_t>(pp * p.D);  // L * D < 2^31 (checked on the host)
             if (umode == 2) {
                 bulk_g2s(smem + Lay::OFF_U + st * Lay::ROWS + r * Lay::ROW, gu + (b * p.L + pp) * p.D + d0,
                          row_bytes, &full[st]);
@@ -647,7 +648,9 @@ __global__ void __launch_bounds__(32 * WARPS)
             const io_t* su = reinterpret_cast<const io_t*>(smem + Lay::OFF_U + st * Lay::ROWS);
             const io_t* sdl = reinterpret_cast<const io_t*>(smem + Lay::OFF_DL + st * Lay::ROWS);
             const io_t* sz = reinterpret_cast<const io_t*>(smem + Lay::OFF_Z + st * Lay::ROWS);
-            const int64_t* orow = reinterpret_cast<const int64_t*>(smem + Lay::OFF_OUT + st * Lay::OUT_STRIDE);
+            const int32_t* orow = reinterpret_cast<const int32_t*>(smem + Lay::OFF_OUT + st * Lay::OUT_STRIDE);
+            float* yp_out = p.ypart ? p.ypart + out_base + tid : nullptr;
+            io_t* o_out = static_cast<io_t*>(p.out) + out_base + tid;
             const float* bf = reinterpret_cast<const float*>(smem + Lay::OFF_BF + st * Lay::BF_STRIDE);
             const float4* B4 = reinterpret_cast<const float4*>(bf);
             const float4* C4 = reinterpret_cast<const float4*>(bf + kTile * NS);
@@ -687,13 +690,13 @@ __global__ void __launch_bounds__(32 * WARPS)
                     if (!PHASE1) {
                         float y = fmaf(dskip, uv, yp);
                         if (YPART) {
-                            p.ypart[orow[r] + tid] = y;
+                            yp_out[orow[r]] = y;
                         } else {
                             if (GATE) {
                                 const float zv = Io<io_t>::ld(sz + (r ^ xmask) * DC + tid);
                                 y *= zv / (1.f + ex2(-zv * kLog2e));
                             }
-                            static_cast<io_t*>(p.out)[orow[r] + tid] = Io<io_t>::st(y);
+                            o_out[orow[r]] = Io<io_t>::st(y);
                         }
                     }
                 }
@@ -702,13 +705,14 @@ __global__ void __launch_bounds__(32 * WARPS)
                 // rows, then their state updates; no branch inside a group, so the compiler can
                 // overlap consecutive rows.  A row past the tile's end leaves the state as it
                 // is: q = 1, w = the previous w (so w_prev/w = 1), and B = 0 there.
-                auto group = [&](auto chain_tag, int r0) {
+                auto group = [&](auto chain_tag, auto full_tag, int r0) {
                     constexpr bool CHAIN = decltype(chain_tag)::value;
+                    constexpr bool FULL = decltype(full_tag)::value;  // all kGroup rows valid
                     float s_q[kGroup], s_w[kGroup], s_rr[kGroup], s_sp[kGroup], s_du[kGroup],
                         s_g[kGroup];
 #pragma unroll
                     for (int g = 0; g < kGroup; ++g) {
-                        const bool valid = r0 + g < rows;
+                        const bool valid = FULL || r0 + g < rows;
                         const int r = valid ? (r0 + g) : (rows - 1);
                         const float uv = Io<io_t>::ld(su + (r ^ xmask) * DC + tid);
                         const float dr = Io<io_t>::ld(sdl + r * DC + tid);
@@ -728,9 +732,9 @@ __global__ void __launch_bounds__(32 * WARPS)
                         s_du[g] = dskip * uv;
                         s_g[g] = 1.f;
                         if (GATE) {
-                            // silu(z) = z * sigmoid(z), sigmoid(z) = (1 + tanh(z/2)) / 2
-                            const float zv = Io<io_t>::ld(sz + (r ^ xmask) * DC + tid);
-                            s_g[g] = zv * fmaf(0.5f, tanh_approx(0.5f * zv), 0.5f);
+                            // silu(z) = z * sigmoid(z) = h + h * tanh(h) with h = z/2
+                            const float hz = 0.5f * Io<io_t>::ld(sz + (r ^ xmask) * DC + tid);
+                            s_g[g] = fmaf(hz, tanh_approx(hz), hz);
                         }
                     }
 #pragma unroll
@@ -789,21 +793,26 @@ __global__ void __launch_bounds__(32 * WARPS)
                             float y = fmaf(s_w[g], ys.x + ys.y, s_du[g]);
                             if (r < rows) {
                                 if (YPART) {
-                                    p.ypart[orow[r] + tid] = y;
+                                    yp_out[orow[r]] = y;
                                 } else {
                                     if (GATE)
                                         y *= s_g[g];
-                                    static_cast<io_t*>(p.out)[orow[r] + tid] = Io<io_t>::st(y);
+                                    o_out[orow[r]] = Io<io_t>::st(y);
                                 }
                             }
                         }
                     }
                 };
                 for (int r0 = 0; r0 < rows; r0 += kGroup) {
-                    if (use_chain)
-                        group(std::true_type{}, r0);
-                    else
-                        group(std::false_type{}, r0);
+                    const bool full_group = r0 + kGroup <= rows;  // the same for the whole CTA
+                    if (use_chain) {
+                        if (full_group)
+                            group(std::true_type{}, std::true_type{}, r0);
+                        else
+                            group(std::true_type{}, std::false_type{}, r0);
+                    } else {
+                        group(std::false_type{}, std::false_type{}, r0);
+                    }
                 }
             }
         }
