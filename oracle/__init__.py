@@ -19,6 +19,10 @@ Readings of the pages that the oracle fixes (each is listed with its reason in t
     as the same gate.
   * With several directions every direction adds its own Dskip*u (each is a full S6 scan).
   * The state starts at zero unless an initial state is given.
+  * With a convolution given, each direction convolves u along its own scan order (causal,
+    depthwise, zero before the first step; the last tap takes the current step) and applies
+    SiLU; the result replaces u in both the Bbar*u term and the D skip ("Understanding Mamba
+    from zero" sec. 6.2 Step 2 and sec. 8; "Vision Mamba" sec. 2.2).
 """
 
 from __future__ import annotations
@@ -60,7 +64,10 @@ def _load():
             lib.ss_oracle_scan.restype = ctypes.c_int
             lib.ss_oracle_scan.argtypes = [i64, i64, i64, i64, i32, dp, i64, i64,
                                            dp, dp, dp, dp, dp, dp, dp, dp,
-                                           i32, i32, dp, dp, i32, dp]
+                                           i32, i32, dp, dp, i32, dp, dp, dp, i64]
+            lib.ss_oracle_conv_silu.restype = ctypes.c_int
+            lib.ss_oracle_conv_silu.argtypes = [i64, i64, i64, i32, dp, i64, i64, dp, dp, dp,
+                                                i64, dp]
             lib.ss_oracle_position.restype = ctypes.c_int64
             lib.ss_oracle_position.argtypes = [i32, i64, i64, i64, i64]
             lib.ss_oracle_max_threads.restype = ctypes.c_int
@@ -86,19 +93,45 @@ def _ptr(x):
     return None if x is None else x.ctypes.data_as(ctypes.c_void_p)
 
 
+def _check_conv(conv_weight, conv_bias, K, D):
+    if conv_weight.ndim != 3 or conv_weight.shape[:2] != (K, D) or conv_weight.shape[2] < 1:
+        raise ValueError("conv_weight must be [K, D, width]")
+    if conv_bias is not None and conv_bias.shape != (K, D):
+        raise ValueError("conv_bias must be [K, D]")
+
+
+def conv_silu(u, conv_weight, conv_bias=None, dirs=(DIR_FORWARD,), H=0, W=0):
+    """The convolved and activated inputs alone: [K, batch, L, D], direction k's scan order."""
+    u, conv_weight, conv_bias = _f64(u), _f64(conv_weight), _f64(conv_bias)
+    dirs_arr = np.ascontiguousarray(np.asarray(dirs, dtype=np.int32).reshape(-1))
+    K = int(dirs_arr.size)
+    batch, L, D = u.shape
+    _check_conv(conv_weight, conv_bias, K, D)
+    out = np.empty((K, batch, L, D), dtype=np.float64)
+    rc = _load().ss_oracle_conv_silu(batch, L, D, K, _ptr(dirs_arr), int(H), int(W), _ptr(u),
+                                     _ptr(conv_weight), _ptr(conv_bias),
+                                     int(conv_weight.shape[2]), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments (code %d)" % rc)
+    return out
+
+
 def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softplus=True,
                    dirs=(DIR_FORWARD,), H=0, W=0, zoh_exact=False, threads=None,
-                   return_last_state=True, initial_state=None):
+                   return_last_state=True, initial_state=None, conv_weight=None,
+                   conv_bias=None):
     """Run the oracle.
 
     u, z: [batch, L, D]; delta: [K, batch, L, D]; B, C: [K, batch, L, N]; A: [D, N];
-    Dskip, delta_bias: [D] or None; initial_state: [K, batch, D, N] or None (zero).  Inputs
-    may be any real dtype; they are upcast to float64 exactly.  Returns (out [batch, L, D],
-    last_state [K, batch, D, N]) in float64.
+    Dskip, delta_bias: [D] or None; initial_state: [K, batch, D, N] or None (zero);
+    conv_weight: [K, D, width] or None (u is used as it is); conv_bias: [K, D] or None.
+    Inputs may be any real dtype; they are upcast to float64 exactly.  Returns
+    (out [batch, L, D], last_state [K, batch, D, N]) in float64.
     """
     u, delta, A, B, C = _f64(u), _f64(delta), _f64(A), _f64(B), _f64(C)
     Dskip, z, delta_bias = _f64(Dskip), _f64(z), _f64(delta_bias)
     initial_state = _f64(initial_state)
+    conv_weight, conv_bias = _f64(conv_weight), _f64(conv_bias)
     dirs_arr = np.ascontiguousarray(np.asarray(dirs, dtype=np.int32).reshape(-1))
     K = int(dirs_arr.size)
     if u.ndim != 3:
@@ -118,6 +151,10 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
             raise ValueError("Dskip and delta_bias must be [D]")
     if initial_state is not None and initial_state.shape != (K, batch, D, N):
         raise ValueError("initial_state must be [K, batch, D, N]")
+    if conv_weight is not None:
+        _check_conv(conv_weight, conv_bias, K, D)
+    elif conv_bias is not None:
+        raise ValueError("conv_bias needs conv_weight")
     out = np.empty((batch, L, D), dtype=np.float64)
     last = np.empty((K, batch, D, N), dtype=np.float64) if return_last_state else None
     if threads is None:
@@ -126,7 +163,8 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
                                 _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip),
                                 _ptr(z), _ptr(delta_bias), int(bool(softplus)),
                                 int(bool(zoh_exact)), _ptr(out), _ptr(last), int(threads),
-                                _ptr(initial_state))
+                                _ptr(initial_state), _ptr(conv_weight), _ptr(conv_bias),
+                                0 if conv_weight is None else int(conv_weight.shape[2]))
     if rc != 0:
         raise ValueError("oracle rejected its arguments (code %d)" % rc)
     return out, last

@@ -12,6 +12,15 @@
  *     h[n] = initial_state[k,b,d,n], or 0 without one     (the state before step 0)
  *     for t = 0 .. L-1:
  *       p     = spatial position visited at step t         (the direction's index map)
+ *       u_t   = u[b,p,d], or, with a convolution given,    ("Understanding Mamba from zero"
+ *               silu(conv_bias[k,d] + sum_j                 sec. 6.2 Step 2: a small depthwise
+ *                 conv_weight[k,d,j] * u[b, p(t-w+1+j), d]) causal 1D conv before the SSM;
+ *               over the taps j = 0..w-1 whose step        width d_conv = 4 in sec. 8; "Vision
+ *               t-w+1+j is >= 0 (zero padding before the    Mamba" sec. 2.2: each direction
+ *               first step), p(s) = position of step s      convolves its own scanned sequence;
+ *                                                          the activation after the conv as in
+ *                                                          Figure 2's caption and the VMamba
+ *                                                          block of "S4 -> Mamba" sec. 3)
  *       Delta = softplus(delta[k,b,t,d] + bias[d])         ("Understanding Mamba from zero",
  *               (or the raw sum when softplus is off)       sec. 4.1 Algorithm 2 / sec. 6.2
  *                                                          Step 3: tau_Delta(Parameter+s_Delta))
@@ -19,10 +28,10 @@
  *              Bbar = Delta * B[k,b,t,n]                   (first-order reading of eq. 4, as on
  *                                                          "Mamba-UNet" sec. 4: Bbar ~ Delta*B)
  *                     or, with zoh_exact, (exp(Delta*A)-1)/A * B   (eq. 4 exactly, diagonal A)
- *              h[n]  = Abar * h[n] + Bbar * u[b,p,d]       (eq. 2a; the per-state scalar
+ *              h[n]  = Abar * h[n] + Bbar * u_t            (eq. 2a; the per-state scalar
  *                                                          recurrence h_t = a_t h_{t-1} + b_t of
  *                                                          sec. 5)
- *       y_k[p] = sum_n C[k,b,t,n] * h[n] + Dskip[d]*u[b,p,d]   (eq. 2b plus the D(t)x(t) skip
+ *       y_k[p] = sum_n C[k,b,t,n] * h[n] + Dskip[d]*u_t    (eq. 2b plus the D(t)x(t) skip
  *                                                          term of "Mamba-UNet" sec. 4)
  *     last_state[k,b,d,n] = h[n] after the last step
  *   out[b,p,d] = (sum_k y_k[p]) * silu(z[b,p,d])          (Step 6 gate phi = SiLU; the Vim block's
@@ -47,6 +56,8 @@
  *   out                  [batch, L, D]
  *   last_state           [K, batch, D, N] or NULL
  *   initial_state        [K, batch, D, N] or NULL (zero)
+ *   conv_weight          [K, D, conv_width] or NULL (no convolution: u_t = u[b,p,d])
+ *   conv_bias            [K, D] or NULL (zero)
  *
  * Parity is pinned by tests/test_oracle_pins.py against the LTI convolution form (eq. 3),
  * Theorem 1, the unrolled double sum, the Delta -> 0 limit, reversal and explicitly permuted
@@ -96,6 +107,50 @@ static double oracle_silu(double v)
     return v / (1.0 + exp(-v));
 }
 
+/* The input of step t of direction dir after the causal depthwise convolution and SiLU: tap j
+ * (0 .. width-1) multiplies the input at step t - (width-1) + j of the same scan order, so the
+ * last tap takes the current step; steps before 0 contribute nothing. */
+static double oracle_conv_silu_step(const double* u, int64_t b, int64_t d, int64_t L, int64_t D,
+                                    int32_t dir, int64_t H, int64_t W, int64_t t,
+                                    const double* w, double bias, int64_t width)
+{
+    double c = bias;
+    for (int64_t j = 0; j < width; ++j) {
+        const int64_t s = t - (width - 1) + j;
+        if (s >= 0)
+            c += w[j] * u[(b * L + ss_oracle_position(dir, L, H, W, s)) * D + d];
+    }
+    return oracle_silu(c);
+}
+
+/* The convolved inputs on their own, for checking: out[k,b,t,d] = u_t of direction k (scan
+ * order).  conv_bias may be NULL. */
+int ss_oracle_conv_silu(int64_t batch, int64_t L, int64_t D, int32_t K, const int32_t* dirs,
+                        int64_t H, int64_t W, const double* u, const double* conv_weight,
+                        const double* conv_bias, int64_t conv_width, double* out)
+{
+    if (batch < 0 || L < 0 || D < 0 || K < 1 || K > 4 || conv_width < 1 || conv_width > 64)
+        return ORACLE_BAD_ARG;
+    if (!u || !conv_weight || !out || !dirs)
+        return ORACLE_BAD_ARG;
+    for (int32_t k = 0; k < K; ++k) {
+        if (dirs[k] < 0 || dirs[k] > 3)
+            return ORACLE_BAD_ARG;
+        if ((dirs[k] == ORACLE_DIR_COLUMN || dirs[k] == ORACLE_DIR_COLUMN_REVERSE) &&
+            (H <= 0 || W <= 0 || H * W != L))
+            return ORACLE_BAD_ARG;
+    }
+    for (int32_t k = 0; k < K; ++k)
+        for (int64_t b = 0; b < batch; ++b)
+            for (int64_t t = 0; t < L; ++t)
+                for (int64_t d = 0; d < D; ++d)
+                    out[(((int64_t)k * batch + b) * L + t) * D + d] = oracle_conv_silu_step(
+                        u, b, d, L, D, dirs[k], H, W, t,
+                        conv_weight + ((int64_t)k * D + d) * conv_width,
+                        conv_bias ? conv_bias[(int64_t)k * D + d] : 0.0, conv_width);
+    return ORACLE_OK;
+}
+
 int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                    const int32_t* dirs, int64_t H, int64_t W,
                    const double* u, const double* delta, const double* A,
@@ -103,10 +158,13 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                    const double* z, const double* delta_bias,
                    int32_t softplus, int32_t zoh_exact,
                    double* out, double* last_state, int32_t nthreads,
-                   const double* initial_state)
+                   const double* initial_state, const double* conv_weight,
+                   const double* conv_bias, int64_t conv_width)
 {
     int bad = 0;
     if (batch < 0 || L < 0 || D < 0 || N < 1 || K < 1 || K > 4)
+        return ORACLE_BAD_ARG;
+    if (conv_weight && (conv_width < 1 || conv_width > 64))
         return ORACLE_BAD_ARG;
     if (!u || !delta || !A || !B || !C || !out || !dirs)
         return ORACLE_BAD_ARG;
@@ -148,7 +206,13 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                                    : 0.0;
                     for (int64_t t = 0; t < L; ++t) {
                         const int64_t p = ss_oracle_position(dirs[k], L, H, W, t);
-                        const double ut = u[(b * L + p) * D + d];
+                        const double ut =
+                            conv_weight
+                                ? oracle_conv_silu_step(
+                                      u, b, d, L, D, dirs[k], H, W, t,
+                                      conv_weight + ((int64_t)k * D + d) * conv_width,
+                                      conv_bias ? conv_bias[(int64_t)k * D + d] : 0.0, conv_width)
+                                : u[(b * L + p) * D + d];
                         const int64_t row = ((int64_t)k * batch + b) * L + t;
                         double dt = delta[row * D + d] + (delta_bias ? delta_bias[d] : 0.0);
                         if (softplus)

@@ -41,6 +41,18 @@ MUTATIONS = [
     ("initial state of the wrong direction", "initial_state[(((int64_t)k * batch + b) * D + d) * N + n]",
      "initial_state[(((int64_t)0 * batch + b) * D + d) * N + n]"),
     ("initial state ignored", "h[n] = initial_state\n", "h[n] = 0 && initial_state\n"),
+    ("conv taps in reverse order", "const int64_t s = t - (width - 1) + j;",
+     "const int64_t s = t - j;"),
+    ("conv along the spatial order", "u[(b * L + ss_oracle_position(dir, L, H, W, s)) * D + d]",
+     "u[(b * L + s) * D + d]"),
+    ("conv bias dropped", "double c = bias;", "double c = 0.0;"),
+    ("no activation after the conv", "return oracle_silu(c);", "return c;"),
+    ("D skip reads the unconvolved input", "(Dskip ? Dskip[d] : 0.0) * ut;",
+     "(Dskip ? Dskip[d] : 0.0) * u[(b * L + p) * D + d];"),
+    ("scan takes conv weights of direction 0", "u, b, d, L, D, dirs[k], H, W, t,\n"
+     "                                      conv_weight + ((int64_t)k * D + d) * conv_width,",
+     "u, b, d, L, D, dirs[k], H, W, t,\n"
+     "                                      conv_weight + ((int64_t)0 * D + d) * conv_width,"),
 ]
 
 
@@ -75,7 +87,8 @@ def test_mutant_fails_a_pin(tmp_path, label, old, new):
                     str(mutant), "-lm"], check=True)
     real = oracle._load()
     lib = ctypes.CDLL(str(so))
-    for fname in ("ss_oracle_scan", "ss_oracle_position", "ss_oracle_max_threads"):
+    for fname in ("ss_oracle_scan", "ss_oracle_position", "ss_oracle_max_threads",
+                  "ss_oracle_conv_silu"):
         getattr(lib, fname).restype = getattr(real, fname).restype
         getattr(lib, fname).argtypes = getattr(real, fname).argtypes
     failed = []

@@ -24,6 +24,13 @@ identity, a special case or a brute force that does not run the oracle's recurre
       the sequence at T, the end state is exp(A * sum Delta_suffix) * h_prefix + h_suffix(0), and
       the suffix outputs gain C_t . (exp(A * partial sums) * h_prefix).
   P8  linearity in u with no gate, and the decay bound |h_n| <= sum_s |Delta_s B_s[n] u_s|.
+  P9  the causal depthwise convolution + SiLU before the scan ("Understanding Mamba from zero"
+      sec. 6.2 Step 2; "Vision Mamba" sec. 2.2, one convolution per scanned sequence) equals
+      numpy's full convolution of each direction's explicitly permuted sequence, truncated to
+      the causal part.
+  P10 a scan with the convolution equals, direction by direction, single scans of the
+      convolved inputs (computed as in P9, put back in spatial order), summed and gated: the
+      convolved value replaces u in both the Bbar*u term and the D skip.
   plus the silu gate against sigmoid written out, a hand-worked Abar = 1/2 example, empty and
   length-1 inputs, and a regression fixture written by tests/golden/make_golden.py.
 """
@@ -426,3 +433,66 @@ def test_P7_initial_state_continues_a_split_scan():
     _, l0 = oracle.selective_scan(e, np.zeros((1, batch, 0, D)), c["A"], np.zeros((1, batch, 0, N)),
                                   np.zeros((1, batch, 0, N)), initial_state=h1)
     assert np.array_equal(l0, h1)
+
+
+# ----------------------------------------------------------------------------- P9, P10 (conv)
+
+def _np_conv_silu(u, w, cb, kind, H, W):
+    """[batch, L, D] in the scan order of `kind`: numpy's convolution of the permuted sequence
+    with the taps reversed (np.convolve flips its kernel), cut to the first L outputs, plus the
+    bias, then x * sigmoid(x)."""
+    order = _perm_by_loops(kind, H, W)
+    seq = u[:, order]
+    L = seq.shape[1]
+    out = np.empty_like(seq)
+    for b in range(seq.shape[0]):
+        for d in range(seq.shape[2]):
+            c = np.convolve(seq[b, :, d], w[d, ::-1])[:L] + cb[d]
+            out[b, :, d] = c / (1.0 + np.exp(-c))
+    return out, order
+
+
+CONV_CASES = [((FWD,), 1, 23, 4), ((FWD, REV), 1, 29, 4), ((FWD, COL, REV, COLREV), 5, 7, 4),
+              ((COLREV, FWD), 3, 4, 2), ((REV,), 1, 9, 1), ((COL,), 4, 3, 3)]
+
+
+@pytest.mark.parametrize("dirs,H,W,width", CONV_CASES)
+def test_P9_conv_equals_numpy_convolution(dirs, H, W, width):
+    rng = np.random.default_rng(40 + width + len(dirs))
+    batch, L, D, K = 2, H * W, 3, len(dirs)
+    u = rng.standard_normal((batch, L, D))
+    w = rng.standard_normal((K, D, width))
+    cb = rng.standard_normal((K, D))
+    got = oracle.conv_silu(u, w, cb, dirs=dirs, H=H, W=W)
+    for k, kind in enumerate(dirs):
+        ref, _ = _np_conv_silu(u, w[k], cb[k], kind, H, W)
+        assert rel_err(got[k], ref) < 1e-13
+    # no bias given reads as zero
+    got0 = oracle.conv_silu(u, w, None, dirs=dirs, H=H, W=W)
+    ref0, _ = _np_conv_silu(u, w[0], np.zeros(D), dirs[0], H, W)
+    assert rel_err(got0[0], ref0) < 1e-13
+
+
+@pytest.mark.parametrize("dirs,H,W,width", CONV_CASES)
+def test_P10_conv_scan_equals_scans_of_convolved_inputs(dirs, H, W, width):
+    rng = np.random.default_rng(60 + width + len(dirs))
+    batch, L, D, N, K = 2, H * W, 3, 4, len(dirs)
+    c = rand_case(rng, batch, L, D, N, K=K)
+    w = rng.standard_normal((K, D, width))
+    cb = rng.standard_normal((K, D))
+    args = dict(Dskip=c["Dskip"], delta_bias=c["delta_bias"], softplus=True)
+    out, last = oracle.selective_scan(c["u"], c["delta"], c["A"], c["B"], c["C"], z=c["z"],
+                                      dirs=dirs, H=H, W=W, conv_weight=w, conv_bias=cb, **args)
+    total = np.zeros_like(c["u"])
+    lasts = []
+    for k, kind in enumerate(dirs):
+        u_scan, order = _np_conv_silu(c["u"], w[k], cb[k], kind, H, W)
+        u_sp = np.empty_like(u_scan)
+        u_sp[:, order] = u_scan                         # the convolved input at its position
+        y_k, l_k = oracle.selective_scan(u_sp, c["delta"][k:k + 1], c["A"], c["B"][k:k + 1],
+                                         c["C"][k:k + 1], z=None, dirs=(kind,), H=H, W=W, **args)
+        total += y_k
+        lasts.append(l_k[0])
+    gate = c["z"] / (1.0 + np.exp(-c["z"]))
+    assert rel_err(out, total * gate) < 1e-12
+    assert rel_err(last, np.stack(lasts)) < 1e-12
