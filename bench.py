@@ -171,7 +171,16 @@ def workload_of(args) -> wl.Workload:
         if w.H:
             raise SystemExit("--seqlen does not apply to image workloads")
         w = wl.variant(w.name, seqlen=args.seqlen)
+    if args.conv:
+        w = wl.variant(w.name, seqlen=w.seqlen, conv=args.conv)
     return w
+
+
+def describe(w: wl.Workload) -> str:
+    text = wl.DESCRIPTIONS[w.name]
+    if w.conv:
+        text += ", causal depthwise conv1d (%d taps) + SiLU fused before the scan" % w.conv
+    return text
 
 
 def workload_bytes(w: wl.Workload) -> int:
@@ -195,7 +204,8 @@ def time_oracle(inp, channels, threads):
     t0 = time.perf_counter()
     oracle.selective_scan(f["u"], f["delta"], f["A"], f["B"], f["C"], Dskip=f["Dskip"], z=f["z"],
                           delta_bias=f["delta_bias"], softplus=w.softplus, dirs=w.dirs, H=w.H,
-                          W=w.W, threads=threads)
+                          W=w.W, threads=threads, conv_weight=f["conv_weight"],
+                          conv_bias=f["conv_bias"])
     return time.perf_counter() - t0
 
 
@@ -227,8 +237,8 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (seeded, %s)" % wl.DESCRIPTIONS[w.name],
-            "config": {"workload": wl.DESCRIPTIONS[w.name], "name": w.name},
+            "data": "synthetic (seeded, %s)" % describe(w),
+            "config": {"workload": describe(w), "name": w.name, "conv": w.conv},
             "updates_per_s": w.updates() * frac / step_s,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": sample},
@@ -243,7 +253,6 @@ def run_reference(args):
 def run_ours(args):
     import torch
     from selective_state_space_13_b200 import scan
-    from tests.scan_util import to_device
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -255,7 +264,7 @@ def run_ours(args):
                                 device_id=device)
     w = workload_of(args)
     inp = wl.make_inputs(w)
-    t = to_device(inp, device)
+    t = wl.to_device(inp, device)
     want_last = w.name in RETURNS_LAST_STATE
     out = torch.empty_like(t["u"])
     last = torch.empty((w.K, w.batch, w.dim, w.dstate), dtype=torch.float32, device=device) \
@@ -267,7 +276,8 @@ def run_ours(args):
         scan.selective_scan_fwd(t["u"], t["delta"], t["A"], t["B"], t["C"], D=t["D"], z=t["z"],
                                 delta_bias=t["delta_bias"], softplus=w.softplus, dirs=w.dirs,
                                 H=w.H, W=w.W, out=out, last_state=last, segments=args.segments,
-                                flags=args.flags, events=events)
+                                flags=args.flags, events=events, conv_weight=t["conv_weight"],
+                                conv_bias=t["conv_bias"])
 
     # plan facts for the report
     shape = scan.make_shape(w.batch, w.seqlen, w.dim, w.dstate,
@@ -381,18 +391,19 @@ def run_ours(args):
                          "(%.3g state updates)" % (len(channels), w.dim, w.seqlen, w.K,
                                                    w.updates() * frac)}
 
-    traffic = recorded_traffic(w.name)
+    traffic = None if args.seqlen else recorded_traffic(
+        w.name + ("_conv%d" % w.conv if w.conv else ""))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == wl.BF16 else "f32",
         "data": "synthetic (seeded N(0,1) inputs, A=-(n+1), log-uniform Delta bias)",
-        "config": {"workload": wl.DESCRIPTIONS[w.name] + (
+        "config": {"workload": describe(w) + (
                        " (seqlen overridden to %d)" % w.seqlen if args.seqlen else ""),
                    "name": w.name, "batch": w.batch,
                    "seqlen": w.seqlen, "dim": w.dim, "dstate": w.dstate, "directions": w.K,
-                   "gate": w.gate, "returns_last_state": want_last,
+                   "gate": w.gate, "returns_last_state": want_last, "conv": w.conv,
                    "parallelism": "independent problems per rank" if world > 1 else "1 GPU",
                    "l2": "flushed (256 MiB write) before every timed step",
                    "segments": args.segments or "auto", "workspace_bytes": ws_bytes},
@@ -435,6 +446,8 @@ def parse(argv=None):
     ap.add_argument("--flags", type=int, default=0, help="SS_FLAG_* bits (1 = generic A)")
     ap.add_argument("--seqlen", type=int, default=0,
                     help="override the workload's sequence length (smaller cases for profiling)")
+    ap.add_argument("--conv", type=int, default=0,
+                    help="taps of a causal depthwise conv1d + SiLU fused before the scan (0 = none)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-updates", type=float, default=4e9,

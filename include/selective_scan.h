@@ -4,6 +4,12 @@
  * The library computes, on one GPU and entirely in its own CUDA kernels, the selective state
  * space scan that the pages describe:
  *
+ *   u_t      = u at the position of step t, or, with a    "Understanding Mamba from zero"
+ *              convolution given (ss_launch_opts),          sec. 6.2 Step 2 (a small depthwise
+ *              silu(conv_bias + sum_j conv_weight[j] *      causal 1D conv before the SSM,
+ *                   u at step t - (width-1) + j)            width 4 in sec. 8); one conv per
+ *              along this direction's scan order, zero      scanned sequence as in "Vision
+ *              before step 0                                Mamba" sec. 2.2
  *   Delta_t  = softplus(delta_raw_t + delta_bias)          "Understanding Mamba from zero",
  *                                                           sec. 4.1 Algorithm 2 and sec. 6.2
  *                                                           Step 3 (tau_Delta(Parameter+s_Delta))
@@ -19,7 +25,8 @@
  *                                                           Mamba" sec. 2.2) and the SS2D merge of
  *                                                           four scan orders ("S4 -> Mamba" sec. 3)
  *
- * with A diagonal (one scalar per channel and state) and the state starting at zero.
+ * with A diagonal (one scalar per channel and state) and the state starting at zero (or at a
+ * given initial state).
  *
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library never frees or
@@ -45,9 +52,10 @@
 extern "C" {
 #endif
 
-#define SS_ABI_VERSION 2
+#define SS_ABI_VERSION 3
 #define SS_MAX_DSTATE 16
 #define SS_MAX_DIRS 4
+#define SS_MAX_CONV_WIDTH 4
 
 typedef enum {
     SS_OK = 0,
@@ -102,7 +110,15 @@ typedef struct {
     const float* initial_state; /* [K, batch, D, N] fp32 device array: the state h before
                                    step 0 of each direction (eq. 2a's h_{-1}), or NULL for
                                    zero; read only; must not overlap last_state             */
-    int32_t reserved[2];     /* must be 0                                                    */
+    const float* conv_weight; /* [K, D, conv_width] fp32 device array: the causal depthwise
+                                 convolution that direction k applies to u along its own scan
+                                 order before the scan, followed by SiLU; tap conv_width-1
+                                 multiplies the current step.  The convolved value replaces u
+                                 in both Bbar*u and the D skip.  NULL: no convolution       */
+    const float* conv_bias;  /* [K, D] fp32 device array, or NULL for zero (needs
+                                conv_weight)                                                 */
+    int32_t conv_width;      /* taps, 1..SS_MAX_CONV_WIDTH with conv_weight; 0 without      */
+    int32_t reserved;        /* must be 0                                                    */
 } ss_launch_opts;
 
 #define SS_FLAG_GENERIC_A 1 /* never use the exp-power shortcut for A[d,n] = (n+1)*A[d,0]   */

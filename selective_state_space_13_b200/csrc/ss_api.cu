@@ -32,6 +32,9 @@ struct Plan {
     int flags;
     cudaEvent_t ev_begin, ev_end;
     const float* init_state;
+    const float* conv_w;
+    const float* conv_b;
+    int conv_width;
     // workspace layout (byte offsets, 0 size = unused)
     size_t off_carry_h, off_carry_s, off_ypart, bytes;
 };
@@ -101,10 +104,20 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
     pl->flags = 0;
     pl->ev_begin = pl->ev_end = nullptr;
     pl->init_state = nullptr;
+    pl->conv_w = pl->conv_b = nullptr;
+    pl->conv_width = 0;
     if (opts) {
-        for (int i = 0; i < 2; ++i)
-            if (opts->reserved[i] != 0)
+        if (opts->reserved != 0)
+            return SS_ERR_UNSUPPORTED;
+        if (opts->conv_weight) {
+            if (opts->conv_width < 1 || opts->conv_width > SS_MAX_CONV_WIDTH)
                 return SS_ERR_UNSUPPORTED;
+        } else if (opts->conv_bias || opts->conv_width != 0) {
+            return SS_ERR_UNSUPPORTED;
+        }
+        pl->conv_w = opts->conv_weight;
+        pl->conv_b = opts->conv_bias;
+        pl->conv_width = opts->conv_weight ? opts->conv_width : 0;
         if (opts->segments < 0 || opts->segments > kMaxSegments)
             return SS_ERR_UNSUPPORTED;
         if (opts->flags & ~(SS_FLAG_GENERIC_A | SS_FLAG_ZOH_EXACT | SS_FLAG_TEST_WAIT_TIMEOUT))
@@ -204,7 +217,8 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
             return SS_ERR_ALIGN;
     for (const void* p : {static_cast<const void*>(A), static_cast<const void*>(Dskip),
                           static_cast<const void*>(delta_bias), static_cast<const void*>(last_state),
-                          static_cast<const void*>(pl.init_state)})
+                          static_cast<const void*>(pl.init_state),
+                          static_cast<const void*>(pl.conv_w), static_cast<const void*>(pl.conv_b)})
         if (p && !aligned(p, 4))
             return SS_ERR_ALIGN;
     if (pl.bytes > 0 && (!workspace || workspace_bytes < pl.bytes))
@@ -257,6 +271,9 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
     p.zoh = (pl.flags & SS_FLAG_ZOH_EXACT) ? 1 : 0;
     p.test_timeout = (pl.flags & SS_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
     p.init_state = pl.init_state;
+    p.conv_w = pl.conv_w;
+    p.conv_b = pl.conv_b;
+    p.conv_width = pl.conv_width;
 
     // the timing events bracket the scan pipeline: the segment-aggregate launch (if any) and
     // the scan launch, which may overlap (nothing is recorded between them)

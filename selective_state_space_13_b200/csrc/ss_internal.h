@@ -34,6 +34,8 @@ struct ScanParams {
     float* ypart;           // [K, batch, L, D] fp32 per-direction outputs (several directions)
     float* last_state;      // [K, batch, D, N] or null
     const float* init_state;  // [K, batch, D, N] state before step 0, or null (zero)
+    const float* conv_w;    // [K, D, conv_width] causal conv taps per direction, or null
+    const float* conv_b;    // [K, D] conv bias, or null (zero)
     float* carry_h;         // [K, batch, S, D, N] end state of each segment scanned from zero
     float* carry_s;         // [K, batch, S, D] sum over the segment of Delta*log2(e)
     int64_t batch, L, D;
@@ -46,6 +48,7 @@ struct ScanParams {
     int32_t col3d;          // 1: column orders load through tm_u3 / tm_z3 (H % 8 == 0)
     int32_t zoh;            // 1: Bbar = (exp(Delta*A) - 1) / A * B (precise arithmetic)
     int32_t test_timeout;   // 1: test hook, wait on a barrier nothing completes and report
+    int32_t conv_width;     // taps of conv_w (1..SS_MAX_CONV_WIDTH) when conv_w is set
 };
 
 struct MergeParams {

@@ -28,6 +28,7 @@ SS_FLAG_TEST_WAIT_TIMEOUT = 8
 SS_ERR_DEVICE_TIMEOUT = 9
 SS_MAX_DSTATE = 16
 SS_MAX_DIRS = 4
+SS_MAX_CONV_WIDTH = 4
 
 STATUS_NAMES = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE",
                 4: "SS_ERR_ALIGN", 5: "SS_ERR_DIRMAP", 6: "SS_ERR_UNSUPPORTED", 7: "SS_ERR_CUDA",
@@ -53,7 +54,9 @@ class SsDirectionMap(ctypes.Structure):
 class SsLaunchOpts(ctypes.Structure):
     _fields_ = [("segments", ctypes.c_int32), ("flags", ctypes.c_int32),
                 ("scan_begin_event", ctypes.c_void_p), ("scan_end_event", ctypes.c_void_p),
-                ("initial_state", ctypes.c_void_p), ("reserved", ctypes.c_int32 * 2)]
+                ("initial_state", ctypes.c_void_p), ("conv_weight", ctypes.c_void_p),
+                ("conv_bias", ctypes.c_void_p), ("conv_width", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class ScanError(RuntimeError):
@@ -154,14 +157,19 @@ def make_dirmap(dirs=(SS_DIR_FWD,), H=0, W=0) -> SsDirectionMap:
     return m
 
 
-def make_opts(segments=0, flags=0, events=None, initial_state=0) -> SsLaunchOpts:
+def make_opts(segments=0, flags=0, events=None, initial_state=0, conv_weight=0, conv_bias=0,
+              conv_width=0) -> SsLaunchOpts:
     """events: optional (begin, end) torch.cuda.Event pair, recorded by the library around its
     main scan launch on the call's stream (each must have been recorded once before, so that
     its CUDA event exists).  initial_state: device address of a [K, batch, D, N] fp32 array
-    (0 = zero state)."""
+    (0 = zero state).  conv_weight / conv_bias: device addresses of the [K, D, conv_width] and
+    [K, D] fp32 causal-convolution taps and bias (0 = none)."""
     o = SsLaunchOpts()
     o.segments, o.flags = int(segments), int(flags)
     o.initial_state = int(initial_state) or None
+    o.conv_weight = int(conv_weight) or None
+    o.conv_bias = int(conv_bias) or None
+    o.conv_width = int(conv_width)
     if events is not None:
         o.scan_begin_event = int(events[0].cuda_event) or None
         o.scan_end_event = int(events[1].cuda_event) or None
@@ -267,7 +275,8 @@ def _workspace(nbytes, device):
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                        dirs=(SS_DIR_FWD,), H=0, W=0, out=None, last_state=None,
                        return_last_state=False, workspace=None, stream=None, segments=0,
-                       flags=0, events=None, initial_state=None, zoh_exact=False):
+                       flags=0, events=None, initial_state=None, zoh_exact=False,
+                       conv_weight=None, conv_bias=None):
     """Selective scan forward on CUDA tensors.
 
     u, z: [batch, L, D]; delta: [K, batch, L, D] (or [batch, L, D] when K = 1); B, C:
@@ -275,6 +284,9 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     u, delta, B, C, z share one dtype (float32 or bfloat16); out has that dtype.
     initial_state: [K, batch, D, N] float32 state before step 0 (None = zero); zoh_exact: use
     Bbar = (exp(Delta*A) - 1) / A * B instead of Delta*B.
+    conv_weight: [K, D, width] float32 (width <= 4), the causal depthwise convolution each
+    direction applies to u along its own scan order, followed by SiLU (None = no convolution);
+    conv_bias: [K, D] float32 or None.
     Returns out, or (out, last_state [K, batch, D, N] float32) with return_last_state.
     """
     import torch
@@ -307,11 +319,21 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
         last_state = torch.empty((K, batch, Dm, N), dtype=torch.float32, device=device)
     _check(last_state, "last_state", (K, batch, Dm, N), torch.float32, device)
     _check(initial_state, "initial_state", (K, batch, Dm, N), torch.float32, device)
+    width = 0
+    if conv_weight is not None:
+        if conv_weight.dim() != 3:
+            raise ValueError("conv_weight must be [K, D, width]")
+        width = int(conv_weight.shape[2])
+        _check(conv_weight, "conv_weight", (K, Dm, width), torch.float32, device)
+    elif conv_bias is not None:
+        raise ValueError("conv_bias needs conv_weight")
+    _check(conv_bias, "conv_bias", (K, Dm), torch.float32, device)
     if zoh_exact:
         flags = int(flags) | SS_FLAG_ZOH_EXACT
     shape = make_shape(batch, L, Dm, N, _io_code(io))
     dmap = make_dirmap(dirs, H, W)
-    opts = make_opts(segments, flags, events, _ptr(initial_state))
+    opts = make_opts(segments, flags, events, _ptr(initial_state), _ptr(conv_weight),
+                     _ptr(conv_bias), width)
     nws = selective_scan_workspace_size(shape, dmap, opts)
     if workspace is None and nws > 0:
         workspace = _workspace(nws, device)

@@ -14,7 +14,11 @@ Recipe (identical for every workload, seed = 20260 + workload index):
   * A[d, n] = -(n + 1) (fp32);
   * Dskip = 1 (fp32), except the tiny workload where Dskip ~ N(0, 1);
   * delta_bias: Delta0 ~ exp(U[ln 1e-3, ln 0.1]) per channel, bias = softplus^-1(Delta0) =
-    Delta0 + log(-expm1(-Delta0)); the tiny workload uses bias = 0.
+    Delta0 + log(-expm1(-Delta0)); the tiny workload uses bias = 0;
+  * with a causal convolution of `conv` taps before the scan (no named workload has one; the
+    variants that test it do): taps and bias per direction and channel ~ U(-1/sqrt(conv),
+    1/sqrt(conv)) in fp32, the usual initial scale of a depthwise convolution of that width
+    (the pages give no weights).
 
 The pages name no dataset for this path; the shapes stand for a Mamba-130M layer (8 x 2048 x
 1536, N = 16), a 131072-token sequence, a Vim-S block (64 images of 14 x 14 patches + a class
@@ -51,6 +55,7 @@ class Workload:
     bias: str = "loguniform"        # "loguniform" or "zero"
     dskip: str = "one"              # "one" or "normal"
     seed: int = 20260
+    conv: int = 0                   # taps of the causal convolution before the scan (0: none)
     extra: dict = field(default_factory=dict, compare=False)
 
     @property
@@ -77,6 +82,8 @@ class Workload:
         nbytes += self.dim * self.dstate * 4 + 2 * self.dim * 4    # A, Dskip, delta_bias
         if with_last_state:
             nbytes += self.K * self.batch * self.dim * self.dstate * 4
+        if self.conv:
+            nbytes += self.K * self.dim * (self.conv + 1) * 4         # conv taps and bias
         return nbytes
 
 
@@ -188,7 +195,14 @@ def make_inputs(w: Workload | str, threads: int | None = None) -> dict:
         d0 = np.exp(g.uniform(math.log(1e-3), math.log(0.1), size=D))
         bias = (d0 + np.log(-np.expm1(-d0))).astype(np.float32)
     A = np.tile(-(np.arange(N, dtype=np.float32) + 1.0), (D, 1))
-    return dict(workload=w, u=u, z=z, delta=delta, B=B, C=C, A=A, Dskip=Dskip, delta_bias=bias)
+    conv_weight = conv_bias = None
+    if w.conv:
+        gc = np.random.Generator(np.random.PCG64(np.random.SeedSequence([root, 6])))
+        lim = 1.0 / math.sqrt(w.conv)
+        conv_weight = gc.uniform(-lim, lim, size=(K, D, w.conv)).astype(np.float32)
+        conv_bias = gc.uniform(-lim, lim, size=(K, D)).astype(np.float32)
+    return dict(workload=w, u=u, z=z, delta=delta, B=B, C=C, A=A, Dskip=Dskip, delta_bias=bias,
+                conv_weight=conv_weight, conv_bias=conv_bias)
 
 
 def inputs_f64(inp: dict, channels=None, batches=None) -> dict:
@@ -213,4 +227,31 @@ def inputs_f64(inp: dict, channels=None, batches=None) -> dict:
                 Dskip=np.asarray(inp["Dskip"][dsel], dtype=np.float64),
                 delta_bias=None if inp["delta_bias"] is None else
                 np.asarray(inp["delta_bias"][dsel], dtype=np.float64),
+                conv_weight=None if inp.get("conv_weight") is None else
+                np.asarray(inp["conv_weight"][:, dsel], dtype=np.float64),
+                conv_bias=None if inp.get("conv_bias") is None else
+                np.asarray(inp["conv_bias"][:, dsel], dtype=np.float64),
                 softplus=w.softplus, dirs=w.dirs, H=w.H, W=w.W)
+
+
+def to_torch(arr, dtype: str, device):
+    """A stored array as a torch tensor on `device` (bf16 bit patterns become bfloat16)."""
+    import torch
+    if arr is None:
+        return None
+    if dtype == BF16 and arr.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(np.ascontiguousarray(arr)).to(device)
+
+
+def to_device(inp: dict, device) -> dict:
+    """The arrays of ``make_inputs`` as torch tensors on `device`, keyed as the binding names
+    its arguments (u, z, delta, B, C, A, D, delta_bias, conv_weight, conv_bias)."""
+    w = inp["workload"]
+    return dict(u=to_torch(inp["u"], w.dtype, device), z=to_torch(inp["z"], w.dtype, device),
+                delta=to_torch(inp["delta"], w.dtype, device), B=to_torch(inp["B"], w.dtype, device),
+                C=to_torch(inp["C"], w.dtype, device), A=to_torch(inp["A"], F32, device),
+                D=to_torch(inp["Dskip"], F32, device),
+                delta_bias=to_torch(inp["delta_bias"], F32, device),
+                conv_weight=to_torch(inp.get("conv_weight"), F32, device),
+                conv_bias=to_torch(inp.get("conv_bias"), F32, device))

@@ -27,23 +27,8 @@ def tol_for(w):
     return TOL_F32 if w.dtype == wl.F32 else TOL_BF16
 
 
-def to_torch(arr, dtype, device):
-    import torch
-    if arr is None:
-        return None
-    if dtype == wl.BF16 and arr.dtype == np.uint16:
-        return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16).to(device)
-    return torch.from_numpy(np.ascontiguousarray(arr)).to(device)
-
-
-def to_device(inp, device):
-    w = inp["workload"]
-    return dict(u=to_torch(inp["u"], w.dtype, device), z=to_torch(inp["z"], w.dtype, device),
-                delta=to_torch(inp["delta"], w.dtype, device), B=to_torch(inp["B"], w.dtype, device),
-                C=to_torch(inp["C"], w.dtype, device), A=to_torch(inp["A"], wl.F32, device),
-                D=to_torch(inp["Dskip"], wl.F32, device),
-                delta_bias=None if inp["delta_bias"] is None else
-                to_torch(inp["delta_bias"], wl.F32, device))
+to_torch = wl.to_torch
+to_device = wl.to_device
 
 
 def out_to_f64(t):
@@ -52,7 +37,7 @@ def out_to_f64(t):
 
 
 def run_gpu(inp, dev_inputs=None, device="cuda:0", segments=0, flags=0, use_z=True, use_D=True,
-            use_bias=True, softplus=None, initial_state=None, zoh_exact=False):
+            use_bias=True, softplus=None, initial_state=None, zoh_exact=False, use_conv_bias=True):
     import torch
     from selective_state_space_13_b200 import scan
     w = inp["workload"]
@@ -64,12 +49,13 @@ def run_gpu(inp, dev_inputs=None, device="cuda:0", segments=0, flags=0, use_z=Tr
         z=t["z"] if use_z else None, delta_bias=t["delta_bias"] if use_bias else None,
         softplus=w.softplus if softplus is None else softplus, dirs=w.dirs, H=w.H, W=w.W,
         return_last_state=True, segments=segments, flags=flags, initial_state=h0,
-        zoh_exact=zoh_exact)
+        zoh_exact=zoh_exact, conv_weight=t.get("conv_weight"),
+        conv_bias=t.get("conv_bias") if use_conv_bias else None)
     return out, last
 
 
 def run_oracle(inp, channels=None, batches=None, use_z=True, use_D=True, use_bias=True,
-               softplus=None, initial_state=None, zoh_exact=False):
+               softplus=None, initial_state=None, zoh_exact=False, use_conv_bias=True):
     w = inp["workload"]
     f = wl.inputs_f64(inp, channels=channels, batches=batches)
     return oracle.selective_scan(f["u"], f["delta"], f["A"], f["B"], f["C"],
@@ -78,4 +64,5 @@ def run_oracle(inp, channels=None, batches=None, use_z=True, use_D=True, use_bia
                                  delta_bias=f["delta_bias"] if use_bias else None,
                                  softplus=w.softplus if softplus is None else softplus,
                                  dirs=w.dirs, H=w.H, W=w.W, initial_state=initial_state,
-                                 zoh_exact=zoh_exact)
+                                 zoh_exact=zoh_exact, conv_weight=f["conv_weight"],
+                                 conv_bias=f["conv_bias"] if use_conv_bias else None)

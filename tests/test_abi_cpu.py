@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol():
     assert set(names) == set(scan.EXPORTED), names
     for name in names:
         assert hasattr(lib, name), name
-    assert scan.ss_abi_version() == 2
+    assert scan.ss_abi_version() == 3
 
 
 def test_status_strings():
@@ -115,6 +115,28 @@ def test_null_alignment_and_workspace_errors():
     o = scan.make_opts(segments=-1)
     with pytest.raises(scan.ScanError):
         scan.selective_scan_workspace_size(sh, None, o)
+    o = scan.make_opts()
+    o.reserved = 1
+    with pytest.raises(scan.ScanError):
+        scan.selective_scan_workspace_size(sh, None, o)
+
+
+def test_conv_options_validated():
+    sh = _shape()
+    ok = scan.make_opts(conv_weight=FAKE, conv_bias=FAKE, conv_width=4)
+    assert scan.selective_scan_workspace_size(sh, None, ok) == 0
+    for bad in (dict(conv_weight=FAKE, conv_width=0), dict(conv_weight=FAKE, conv_width=5),
+                dict(conv_weight=FAKE, conv_width=-1), dict(conv_bias=FAKE),
+                dict(conv_width=4)):
+        with pytest.raises(scan.ScanError) as e:
+            scan.selective_scan_workspace_size(sh, None, scan.make_opts(**bad))
+        assert e.value.status == 6, bad
+    # misaligned taps or bias are refused before any launch
+    for kw in (dict(conv_weight=FAKE + 2, conv_width=4),
+               dict(conv_weight=FAKE, conv_bias=FAKE + 1, conv_width=4)):
+        st = scan.selective_scan_fwd_raw(sh, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, 0, 1, None,
+                                         FAKE, 0, 0, 0, 0, scan.make_opts(**kw))
+        assert st == 4, kw
 
 
 def test_workspace_sizes():

@@ -195,6 +195,51 @@ def test_device_status_clean(cuda_device):
     assert scan.selective_scan_device_status(clear=True) == scan.SS_OK
 
 
+# ----------------------------------------------------------------------------- fused conv
+
+@pytest.mark.parametrize("segments", [0, 1, 3])
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F32])
+def test_conv_single_direction(cuda_device, dtype, segments):
+    w = wl.variant("m130", name="conv1", batch=2, seqlen=300, dim=136, dtype=dtype, conv=4,
+                   seed=120)
+    _check(wl.make_inputs(w), cuda_device, segments=segments)
+
+
+@pytest.mark.parametrize("width", [1, 2, 3])
+def test_conv_narrow_widths(cuda_device, width):
+    w = wl.variant("m130", name="convw", batch=2, seqlen=77, dim=64, conv=width, seed=121 + width)
+    _check(wl.make_inputs(w), cuda_device, segments=2)
+
+
+@pytest.mark.parametrize("segments", [0, 2])
+def test_conv_vim_per_direction(cuda_device, segments):
+    w = wl.variant("vim", name="conv_vim", batch=3, dim=64, conv=4, seed=125)
+    _check(wl.make_inputs(w), cuda_device, segments=segments)
+
+
+@pytest.mark.parametrize("H,W", [(12, 10), (16, 8)])
+def test_conv_cross_scan_orders(cuda_device, H, W):
+    # H % 8 != 0 reads rows one by one, H % 8 == 0 through the 8-row column boxes
+    w = wl.variant("ss2d", name="conv_ss2d", batch=2, seqlen=H * W, H=H, W=W, dim=32, conv=4,
+                   seed=126 + H)
+    _check(wl.make_inputs(w), cuda_device, segments=2)
+
+
+def test_conv_without_bias_and_with_generic_A(cuda_device):
+    w = wl.variant("m130", name="conv_nb", batch=2, seqlen=150, dim=64, conv=4, seed=128)
+    inp = wl.make_inputs(w)
+    rng = np.random.default_rng(10)
+    inp["A"] = (-rng.uniform(0.05, 3.0, size=inp["A"].shape)).astype(np.float32)
+    _check(inp, cuda_device, segments=3, use_conv_bias=False)
+
+
+def test_conv_with_initial_state_and_exact_zoh(cuda_device):
+    w = wl.variant("vim", name="conv_h0", batch=2, seqlen=130, dim=64, conv=4, seed=129)
+    inp = wl.make_inputs(w)
+    h0 = np.random.default_rng(11).standard_normal((w.K, w.batch, w.dim, w.dstate)).astype(np.float32)
+    _check(inp, cuda_device, segments=2, initial_state=h0, zoh_exact=True)
+
+
 # ----------------------------------------------------------------------------- full size
 
 FULL_SAMPLES = {
@@ -204,13 +249,14 @@ FULL_SAMPLES = {
     "long": (None, 64),
     "vim": (8, 32),
     "ss2d": (4, 16),
+    "m130_conv": (None, 24),
 }
 
 
-@pytest.mark.parametrize("name", ["tiny", "m130", "long", "vim", "ss2d"])
+@pytest.mark.parametrize("name", ["tiny", "m130", "long", "vim", "ss2d", "m130_conv"])
 def test_full_size_workloads_sampled(cuda_device, name):
     import torch
-    w = wl.WORKLOADS[name]
+    w = wl.variant("m130", conv=4) if name == "m130_conv" else wl.WORKLOADS[name]
     inp = wl.make_inputs(w)
     t = to_device(inp, cuda_device)
     out, last = run_gpu(inp, dev_inputs=t)            # default launch = the benchmark's
