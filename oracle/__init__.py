@@ -19,6 +19,9 @@ Readings of the pages that the oracle fixes (each is listed with its reason in t
     as the same gate.
   * With several directions every direction adds its own Dskip*u (each is a full S6 scan).
   * The state starts at zero unless an initial state is given.
+  * With u given per direction ([K, batch, L, D]), direction k scans its own input; Sigma's
+    CroMB ("S4 -> Mamba" sec. 4.1) is two such directions in forward order with the C of the
+    other modality, summed.
   * With a convolution given, each direction convolves u along its own scan order (causal,
     depthwise, zero before the first step; the last tap takes the current step) and applies
     SiLU; the result replaces u in both the Bbar*u term and the D skip ("Understanding Mamba
@@ -64,7 +67,7 @@ def _load():
             lib.ss_oracle_scan.restype = ctypes.c_int
             lib.ss_oracle_scan.argtypes = [i64, i64, i64, i64, i32, dp, i64, i64,
                                            dp, dp, dp, dp, dp, dp, dp, dp,
-                                           i32, i32, dp, dp, i32, dp, dp, dp, i64]
+                                           i32, i32, dp, dp, i32, dp, dp, dp, i64, i32]
             lib.ss_oracle_conv_silu.restype = ctypes.c_int
             lib.ss_oracle_conv_silu.argtypes = [i64, i64, i64, i32, dp, i64, i64, dp, dp, dp,
                                                 i64, dp]
@@ -122,7 +125,8 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
                    conv_bias=None):
     """Run the oracle.
 
-    u, z: [batch, L, D]; delta: [K, batch, L, D]; B, C: [K, batch, L, N]; A: [D, N];
+    u, z: [batch, L, D] (u may be [K, batch, L, D]: direction k then reads u[k], as in the
+    cross-modal scan); delta: [K, batch, L, D]; B, C: [K, batch, L, N]; A: [D, N];
     Dskip, delta_bias: [D] or None; initial_state: [K, batch, D, N] or None (zero);
     conv_weight: [K, D, width] or None (u is used as it is); conv_bias: [K, D] or None.
     Inputs may be any real dtype; they are upcast to float64 exactly.  Returns
@@ -134,9 +138,10 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
     conv_weight, conv_bias = _f64(conv_weight), _f64(conv_bias)
     dirs_arr = np.ascontiguousarray(np.asarray(dirs, dtype=np.int32).reshape(-1))
     K = int(dirs_arr.size)
-    if u.ndim != 3:
-        raise ValueError("u must be [batch, L, D]")
-    batch, L, D = u.shape
+    u_per_dir = u.ndim == 4
+    if u.ndim not in (3, 4) or (u_per_dir and u.shape[0] != K):
+        raise ValueError("u must be [batch, L, D] or [K, batch, L, D]")
+    batch, L, D = u.shape[-3:]
     if A.ndim != 2 or A.shape[0] != D:
         raise ValueError("A must be [D, N]")
     N = A.shape[1]
@@ -144,8 +149,8 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
         raise ValueError("delta must be [K, batch, L, D], got %r" % (delta.shape,))
     if B.shape != (K, batch, L, N) or C.shape != (K, batch, L, N):
         raise ValueError("B and C must be [K, batch, L, N]")
-    if z is not None and z.shape != u.shape:
-        raise ValueError("z must match u")
+    if z is not None and z.shape != (batch, L, D):
+        raise ValueError("z must be [batch, L, D]")
     for v in (Dskip, delta_bias):
         if v is not None and v.shape != (D,):
             raise ValueError("Dskip and delta_bias must be [D]")
@@ -164,7 +169,8 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
                                 _ptr(z), _ptr(delta_bias), int(bool(softplus)),
                                 int(bool(zoh_exact)), _ptr(out), _ptr(last), int(threads),
                                 _ptr(initial_state), _ptr(conv_weight), _ptr(conv_bias),
-                                0 if conv_weight is None else int(conv_weight.shape[2]))
+                                0 if conv_weight is None else int(conv_weight.shape[2]),
+                                int(u_per_dir))
     if rc != 0:
         raise ValueError("oracle rejected its arguments (code %d)" % rc)
     return out, last

@@ -38,6 +38,11 @@
  *                                                          sigma(z)*(y_fwd+y_bwd), "Vision Mamba"
  *                                                          sec. 2.2; SS2D merge, "S4 -> Mamba" sec. 3)
  *
+ * With u_per_direction, direction k reads its own input u[k] wherever u appears above.  This is
+ * the cross-modal scan of Sigma's CroMB ("S4 -> Mamba" sec. 4.1): two modalities, each scanned
+ * over its own input with the C of the other modality, outputs summed -- the caller stacks the
+ * inputs as directions and passes C in swapped order.
+ *
  * Direction maps (which spatial position p a scan visits at step t), for a sequence that is an
  * H x W image flattened row by row (raster order, "Understanding Mamba from zero" sec. 7.2):
  *   0 forward:          p = t
@@ -47,7 +52,7 @@
  * Directions 2 and 3 are the two other cross-scan orders of VMamba's SS2D ("S4 -> Mamba" sec. 3).
  *
  * Layouts (row-major, all double):
- *   u, z                 [batch, L, D]   spatial order
+ *   u, z                 [batch, L, D]   spatial order (u: [K, batch, L, D] with u_per_direction)
  *   delta                [K, batch, L, D] scan order of direction k
  *   B, C                 [K, batch, L, N] scan order of direction k
  *   A                    [D, N]
@@ -159,7 +164,7 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                    int32_t softplus, int32_t zoh_exact,
                    double* out, double* last_state, int32_t nthreads,
                    const double* initial_state, const double* conv_weight,
-                   const double* conv_bias, int64_t conv_width)
+                   const double* conv_bias, int64_t conv_width, int32_t u_per_direction)
 {
     int bad = 0;
     if (batch < 0 || L < 0 || D < 0 || N < 1 || K < 1 || K > 4)
@@ -200,6 +205,7 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                 const int64_t b = bd / D, d = bd % D;
                 memset(yacc, 0, sizeof(double) * (size_t)L);
                 for (int32_t k = 0; k < K; ++k) {
+                    const double* uk = u_per_direction ? u + (int64_t)k * batch * L * D : u;
                     for (int64_t n = 0; n < N; ++n)
                         h[n] = initial_state
                                    ? initial_state[(((int64_t)k * batch + b) * D + d) * N + n]
@@ -209,10 +215,10 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                         const double ut =
                             conv_weight
                                 ? oracle_conv_silu_step(
-                                      u, b, d, L, D, dirs[k], H, W, t,
+                                      uk, b, d, L, D, dirs[k], H, W, t,
                                       conv_weight + ((int64_t)k * D + d) * conv_width,
                                       conv_bias ? conv_bias[(int64_t)k * D + d] : 0.0, conv_width)
-                                : u[(b * L + p) * D + d];
+                                : uk[(b * L + p) * D + d];
                         const int64_t row = ((int64_t)k * batch + b) * L + t;
                         double dt = delta[row * D + d] + (delta_bias ? delta_bias[d] : 0.0);
                         if (softplus)

@@ -22,8 +22,10 @@ Recipe (identical for every workload, seed = 20260 + workload index):
 
 The pages name no dataset for this path; the shapes stand for a Mamba-130M layer (8 x 2048 x
 1536, N = 16), a 131072-token sequence, a Vim-S block (64 images of 14 x 14 patches + a class
-token = 197 tokens, D = 768, two directions) and a VMamba stage-1 map (56 x 56, D = 192, four
-cross-scan orders).
+token = 197 tokens, D = 768, two directions), a VMamba stage-1 map (56 x 56, D = 192, four
+cross-scan orders) and a cross-modal (CroMB) scan of two modalities over a 120 x 160 feature map
+(a 480 x 640 RGB-D frame at 1/4 resolution, D = 192): one input per modality (u[k] ~ N(0, 1),
+``SeedSequence([seed, 0, k])``), where C[k] stands for the C computed from the other modality.
 """
 
 from __future__ import annotations
@@ -56,6 +58,7 @@ class Workload:
     dskip: str = "one"              # "one" or "normal"
     seed: int = 20260
     conv: int = 0                   # taps of the causal convolution before the scan (0: none)
+    u_per_dir: bool = False         # one input u[k] per direction ([K, batch, L, D])
     extra: dict = field(default_factory=dict, compare=False)
 
     @property
@@ -76,7 +79,8 @@ class Workload:
         e = self.io_bytes
         bld = self.batch * self.seqlen * self.dim
         bln = self.batch * self.seqlen * self.dstate
-        nbytes = bld * e * (2 + (1 if self.gate else 0))          # u, out, z
+        nbytes = bld * e * ((self.K if self.u_per_dir else 1) + 1 + (1 if self.gate else 0))
+        # u (per direction or shared), out, z
         nbytes += self.K * bld * e                                 # delta_raw per direction
         nbytes += 2 * self.K * bln * e                             # B, C per direction
         nbytes += self.dim * self.dstate * 4 + 2 * self.dim * 4    # A, Dskip, delta_bias
@@ -95,6 +99,8 @@ WORKLOADS = {
     "ss2d": Workload("ss2d", 32, 3136, 192, 16, BF16,
                      dirs=(DIR_FORWARD, DIR_COLUMN, DIR_REVERSE, DIR_COLUMN_REVERSE),
                      H=56, W=56, gate=False, seed=20264),
+    "cromb": Workload("cromb", 8, 19200, 192, 16, BF16, dirs=(DIR_FORWARD, DIR_FORWARD),
+                      gate=False, u_per_dir=True, seed=20265),
 }
 
 DESCRIPTIONS = {
@@ -103,6 +109,8 @@ DESCRIPTIONS = {
     "long": "long-sequence scan: batch 1, L 131072, D 5120, N 16, bf16",
     "vim": "Vim-S bidirectional scan: batch 64, M 197, D 768, N 16, bf16, 2 directions",
     "ss2d": "SS2D cross-scan: batch 32, 56x56 (L 3136), D 192, N 16, bf16, 4 directions, no gate",
+    "cromb": "CroMB cross-modal scan: 2 modalities, batch 8, 120x160 (L 19200), D 192, N 16, bf16, "
+             "outputs summed, no gate",
 }
 
 
@@ -167,7 +175,8 @@ def make_inputs(w: Workload | str, threads: int | None = None) -> dict:
     """Draw the seeded inputs of a workload.
 
     Returns a dict with numpy arrays
-      u, z (z is None without a gate) [batch, L, D]; delta [K, batch, L, D]; B, C [K, batch, L, N]
+      u [batch, L, D] (or [K, batch, L, D] with one input per direction), z (None without a
+      gate) [batch, L, D]; delta [K, batch, L, D]; B, C [K, batch, L, N]
       (uint16 bfloat16 bit patterns or float32), A [D, N], Dskip [D], delta_bias [D] or None
       (float32), plus the workload under key "workload".
     """
@@ -178,7 +187,10 @@ def make_inputs(w: Workload | str, threads: int | None = None) -> dict:
     b, L, D, N, K = w.batch, w.seqlen, w.dim, w.dstate, w.K
     root = w.seed
     ss = lambda tid, k=0: np.random.SeedSequence([root, tid, k])  # noqa: E731
-    u = _normal((b, L, D), ss(0), w.dtype, threads)
+    if w.u_per_dir:
+        u = np.stack([_normal((b, L, D), ss(0, k), w.dtype, threads) for k in range(K)])
+    else:
+        u = _normal((b, L, D), ss(0), w.dtype, threads)
     z = _normal((b, L, D), ss(1), w.dtype, threads) if w.gate else None
     delta = np.stack([_normal((b, L, D), ss(2, k), w.dtype, threads) for k in range(K)]) \
         if K > 1 else _normal((b, L, D), ss(2, 0), w.dtype, threads)[None]
@@ -221,7 +233,7 @@ def inputs_f64(inp: dict, channels=None, batches=None) -> dict:
     def bc(x):
         return to_f64(x[:, bsel], w.dtype)
 
-    return dict(u=big(inp["u"], False), z=big(inp["z"], False), delta=big(inp["delta"], True),
+    return dict(u=big(inp["u"], w.u_per_dir), z=big(inp["z"], False), delta=big(inp["delta"], True),
                 B=bc(inp["B"]), C=bc(inp["C"]),
                 A=np.asarray(inp["A"][dsel], dtype=np.float64),
                 Dskip=np.asarray(inp["Dskip"][dsel], dtype=np.float64),

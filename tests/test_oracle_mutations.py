@@ -49,10 +49,12 @@ MUTATIONS = [
     ("no activation after the conv", "return oracle_silu(c);", "return c;"),
     ("D skip reads the unconvolved input", "(Dskip ? Dskip[d] : 0.0) * ut;",
      "(Dskip ? Dskip[d] : 0.0) * u[(b * L + p) * D + d];"),
-    ("scan takes conv weights of direction 0", "u, b, d, L, D, dirs[k], H, W, t,\n"
+    ("scan takes conv weights of direction 0", "uk, b, d, L, D, dirs[k], H, W, t,\n"
      "                                      conv_weight + ((int64_t)k * D + d) * conv_width,",
-     "u, b, d, L, D, dirs[k], H, W, t,\n"
+     "uk, b, d, L, D, dirs[k], H, W, t,\n"
      "                                      conv_weight + ((int64_t)0 * D + d) * conv_width,"),
+    ("every direction reads the first input", "u_per_direction ? u + (int64_t)k * batch",
+     "u_per_direction ? u + (int64_t)0 * batch"),
 ]
 
 

@@ -31,6 +31,10 @@ identity, a special case or a brute force that does not run the oracle's recurre
   P10 a scan with the convolution equals, direction by direction, single scans of the
       convolved inputs (computed as in P9, put back in spatial order), summed and gated: the
       convolved value replaces u in both the Bbar*u term and the D skip.
+  P11 with an input per direction, a K-direction scan equals the sum of K single-direction
+      scans of those inputs, gated; and Sigma's CroMB ("S4 -> Mamba" sec. 4.1) written as the
+      pages give it, SSM(x_rgb, C=C_depth) + SSM(x_depth, C=C_rgb) from two separate scans,
+      equals the two-direction scan with the C tensors stacked in swapped order.
   plus the silu gate against sigmoid written out, a hand-worked Abar = 1/2 example, empty and
   length-1 inputs, and a regression fixture written by tests/golden/make_golden.py.
 """
@@ -496,3 +500,51 @@ def test_P10_conv_scan_equals_scans_of_convolved_inputs(dirs, H, W, width):
     gate = c["z"] / (1.0 + np.exp(-c["z"]))
     assert rel_err(out, total * gate) < 1e-12
     assert rel_err(last, np.stack(lasts)) < 1e-12
+
+
+# ----------------------------------------------------------------------------- P11 (input per direction)
+
+@pytest.mark.parametrize("dirs,H,W,width", [((FWD, COL, REV, COLREV), 5, 7, 0),
+                                            ((FWD, REV), 1, 19, 4), ((FWD, FWD), 1, 23, 0),
+                                            ((COL, FWD, REV), 4, 6, 3)])
+def test_P11_input_per_direction_is_a_sum_of_scans(dirs, H, W, width):
+    rng = np.random.default_rng(80 + len(dirs) + width)
+    batch, L, D, N, K = 2, H * W, 3, 4, len(dirs)
+    c = rand_case(rng, batch, L, D, N, K=K)
+    u = rng.standard_normal((K, batch, L, D))
+    conv = {}
+    if width:
+        conv = dict(conv_weight=rng.standard_normal((K, D, width)),
+                    conv_bias=rng.standard_normal((K, D)))
+    args = dict(Dskip=c["Dskip"], delta_bias=c["delta_bias"], softplus=True, H=H, W=W)
+    out, last = oracle.selective_scan(u, c["delta"], c["A"], c["B"], c["C"], z=c["z"], dirs=dirs,
+                                      **conv, **args)
+    total = np.zeros((batch, L, D))
+    lasts = []
+    for k, kind in enumerate(dirs):
+        conv_k = {key: v[k:k + 1] for key, v in conv.items()}
+        y_k, l_k = oracle.selective_scan(u[k], c["delta"][k:k + 1], c["A"], c["B"][k:k + 1],
+                                         c["C"][k:k + 1], z=None, dirs=(kind,), **conv_k, **args)
+        total += y_k
+        lasts.append(l_k[0])
+    gate = c["z"] / (1.0 + np.exp(-c["z"]))
+    assert rel_err(out, total * gate) < 1e-13
+    assert np.array_equal(last, np.stack(lasts))
+
+
+def test_P11_cromb_cross_modal_scan():
+    rng = np.random.default_rng(90)
+    batch, L, D, N = 2, 31, 4, 5
+    x_rgb, x_depth = rng.standard_normal((2, batch, L, D))
+    d_rgb, d_depth = rng.standard_normal((2, 1, batch, L, D))
+    B_rgb, B_depth, C_rgb, C_depth = rng.standard_normal((4, 1, batch, L, N))
+    A = -rng.uniform(0.1, 2.0, size=(D, N))
+    Dskip = rng.standard_normal(D)
+    bias = rng.uniform(-2.0, 0.5, size=D)
+    args = dict(Dskip=Dskip, delta_bias=bias, softplus=True, z=None)
+    out_rgb, _ = oracle.selective_scan(x_rgb, d_rgb, A, B_rgb, C_depth, **args)
+    out_depth, _ = oracle.selective_scan(x_depth, d_depth, A, B_depth, C_rgb, **args)
+    out, _ = oracle.selective_scan(np.stack([x_rgb, x_depth]), np.concatenate([d_rgb, d_depth]), A,
+                                   np.concatenate([B_rgb, B_depth]),
+                                   np.concatenate([C_depth, C_rgb]), dirs=(FWD, FWD), **args)
+    assert rel_err(out, out_rgb + out_depth) < 1e-13
