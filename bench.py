@@ -266,7 +266,7 @@ def run_ours(args):
     inp = wl.make_inputs(w)
     t = wl.to_device(inp, device)
     want_last = w.name in RETURNS_LAST_STATE
-    out = torch.empty_like(t["u"])
+    out = torch.empty((w.batch, w.seqlen, w.dim), dtype=t["u"].dtype, device=device)
     last = torch.empty((w.K, w.batch, w.dim, w.dstate), dtype=torch.float32, device=device) \
         if want_last else None
     stream = torch.cuda.current_stream(device)

@@ -125,6 +125,12 @@ typedef struct {
 #define SS_FLAG_ZOH_EXACT 2 /* Bbar = (exp(Delta*A) - 1) / A * B, eq. (4) exactly (A != 0;
                                Delta*B where A == 0), instead of the first-order Delta*B;
                                computed with the precise arithmetic for any io type        */
+#define SS_FLAG_U_PER_DIRECTION 16 /* u is [K, batch, L, D]: direction k scans its own input
+                                      u[k] (spatial order), in the convolution too; z stays
+                                      [batch, L, D].  Sigma's cross-modal scan (CroMB, "S4 ->
+                                      Mamba" sec. 4.1) is two forward directions over the two
+                                      modalities' inputs with the C tensors stacked in swapped
+                                      order, so that each modality reads the other's C      */
 #define SS_FLAG_TEST_WAIT_TIMEOUT 8 /* test hook for failure detection: every CTA waits (20 ms
                                        at most) on a barrier that nothing completes, gives up,
                                        records SS_ERR_DEVICE_TIMEOUT for
@@ -141,7 +147,8 @@ ss_status selective_scan_workspace_size(const ss_shape* shape, const ss_directio
  * The selective scan forward (see the top of this file for what it computes).
  *
  *   shape       problem sizes and io dtype (host pointer)
- *   u           [batch, L, D]      io dtype, spatial order
+ *   u           [batch, L, D]      io dtype, spatial order ([K, batch, L, D] with
+ *                                  SS_FLAG_U_PER_DIRECTION)
  *   delta       [K, batch, L, D]   io dtype, raw Delta of direction k in its scan order
  *   A           [D, N]             fp32, shared by all directions
  *   B, C        [K, batch, L, N]   io dtype, scan order of direction k

@@ -120,7 +120,8 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
         pl->conv_width = opts->conv_weight ? opts->conv_width : 0;
         if (opts->segments < 0 || opts->segments > kMaxSegments)
             return SS_ERR_UNSUPPORTED;
-        if (opts->flags & ~(SS_FLAG_GENERIC_A | SS_FLAG_ZOH_EXACT | SS_FLAG_TEST_WAIT_TIMEOUT))
+        if (opts->flags & ~(SS_FLAG_GENERIC_A | SS_FLAG_ZOH_EXACT | SS_FLAG_TEST_WAIT_TIMEOUT |
+                            SS_FLAG_U_PER_DIRECTION))
             return SS_ERR_UNSUPPORTED;
         pl->init_state = opts->initial_state;
         seg = opts->segments;
@@ -270,6 +271,7 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
     p.force_generic = (pl.flags & SS_FLAG_GENERIC_A) ? 1 : 0;
     p.zoh = (pl.flags & SS_FLAG_ZOH_EXACT) ? 1 : 0;
     p.test_timeout = (pl.flags & SS_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
+    p.u_per_dir = (pl.flags & SS_FLAG_U_PER_DIRECTION) ? 1 : 0;
     p.init_state = pl.init_state;
     p.conv_w = pl.conv_w;
     p.conv_b = pl.conv_b;

@@ -22,7 +22,7 @@ struct ScanParams {
     CUtensorMap tm_u, tm_z;    // u, z as [batch*L rows, D]: boxes of kTile rows x DC channels
     CUtensorMap tm_dl;         // delta as [K*batch*L rows, D], same boxes
     CUtensorMap tm_u3, tm_z3;  // u, z as [batch*H, W, D]: boxes of 8 image rows of one column
-    const void* u;          // [batch, L, D] io, spatial order
+    const void* u;          // [batch, L, D] io, spatial order ([K, batch, L, D] with u_per_dir)
     const void* delta;      // [K, batch, L, D] io, scan order
     const float* A;         // [D, N]
     const void* B;          // [K, batch, L, N] io, scan order
@@ -49,6 +49,7 @@ struct ScanParams {
     int32_t zoh;            // 1: Bbar = (exp(Delta*A) - 1) / A * B (precise arithmetic)
     int32_t test_timeout;   // 1: test hook, wait on a barrier nothing completes and report
     int32_t conv_width;     // taps of conv_w (1..SS_MAX_CONV_WIDTH) when conv_w is set
+    int32_t u_per_dir;      // 1: direction k reads its own input u[k]
 };
 
 struct MergeParams {

@@ -358,6 +358,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     const io_t* gB = static_cast<const io_t*>(p.B);
     const io_t* gC = static_cast<const io_t*>(p.C);
     const int64_t kb = static_cast<int64_t>(k) * p.batch + b;  // (direction, batch) row block
+    const int64_t ub = p.u_per_dir ? kb : b;                   // row block of this CTA's u
     // output rows: out[b, p, :] for one direction, ypart[k, b, p, :] for several; a row's
     // element offset from this CTA's base (row 0 of its block, channel d0) fits in 32 bits
     const int64_t out_base = (p.ypart ? kb * p.L : b * p.L) * p.D + d0;
@@ -432,12 +433,12 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
                    static_cast<int32_t>(kb * p.L + t0), &full[st]);
             if (umode == 0) {
                 // reverse order: the box ends at the row of step t0
-                const int64_t prow = b * p.L + (dir == SS_DIR_FWD ? t0 : p.L - t0 - kTile);
+                const int64_t prow = (dir == SS_DIR_FWD ? t0 : p.L - t0 - kTile);
                 tma_2d(smem + Lay::OFF_U + st * Lay::ROWS, &p.tm_u, static_cast<int32_t>(d0),
-                       static_cast<int32_t>(prow), &full[st]);
+                       static_cast<int32_t>(ub * p.L + prow), &full[st]);
                 if (Lay::HAS_Z)
                     tma_2d(smem + Lay::OFF_Z + st * Lay::ROWS, &p.tm_z, static_cast<int32_t>(d0),
-                           static_cast<int32_t>(prow), &full[st]);
+                           static_cast<int32_t>(b * p.L + prow), &full[st]);
             } else if (umode == 1) {
                 for (int sub = 0; sub < rows / 8; ++sub) {
                     const int64_t tt = t0 + 8 * sub;
@@ -446,7 +447,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
                     const int64_t j = c / p.H, i = c - (c / p.H) * p.H;
                     tma_3d(smem + Lay::OFF_U + st * Lay::ROWS + 8 * sub * Lay::ROW, &p.tm_u3,
                            static_cast<int32_t>(d0), static_cast<int32_t>(j),
-                           static_cast<int32_t>(b * p.H + i), &full[st]);
+                           static_cast<int32_t>(ub * p.H + i), &full[st]);
                     if (Lay::HAS_Z)
                         tma_3d(smem + Lay::OFF_Z + st * Lay::ROWS + 8 * sub * Lay::ROW, &p.tm_z3,
                                static_cast<int32_t>(d0), static_cast<int32_t>(j),
@@ -463,7 +464,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
             const int64_t pp = position(dir, p.L, p.H, p.W, t0 + r);
             orow[r] = static_cast<int32_t>(pp * p.D);  // L * D < 2^31 (checked on the host)
             if (umode == 2) {
-                bulk_g2s(smem + Lay::OFF_U + st * Lay::ROWS + r * Lay::ROW, gu + (b * p.L + pp) * p.D + d0,
+                bulk_g2s(smem + Lay::OFF_U + st * Lay::ROWS + r * Lay::ROW, gu + (ub * p.L + pp) * p.D + d0,
                          row_bytes, &full[st]);
                 if (Lay::HAS_Z)
                     bulk_g2s(smem + Lay::OFF_Z + st * Lay::ROWS + r * Lay::ROW, gz + (b * p.L + pp) * p.D + d0,
@@ -562,7 +563,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
         }
         cbias = p.conv_b ? 0.5f * p.conv_b[static_cast<int64_t>(k) * p.D + d] : 0.f;
         auto halo = [&](int64_t t) {
-            return t >= 0 ? Io<io_t>::ld(gu + (b * p.L + position(dir, p.L, p.H, p.W, t)) * p.D + d)
+            return t >= 0 ? Io<io_t>::ld(gu + (ub * p.L + position(dir, p.L, p.H, p.W, t)) * p.D + d)
                           : 0.f;
         };
         xm1 = halo(t_begin - 1);
@@ -1023,7 +1024,9 @@ cudaError_t make_maps(ScanParams& p, bool need_z)
     const cuuint64_t pitch2[1] = {D * esz};
     const cuuint64_t dims_bl[2] = {D, static_cast<cuuint64_t>(p.batch * p.L)};
     const cuuint64_t dims_kbl[2] = {D, static_cast<cuuint64_t>(p.K * p.batch * p.L)};
-    if (!encode(&p.tm_u, p.u, bf16, 2, dims_bl, pitch2, box2) ||
+    const int64_t u_blocks = p.u_per_dir ? p.K * p.batch : p.batch;  // row blocks of u
+    const cuuint64_t dims_u[2] = {D, static_cast<cuuint64_t>(u_blocks * p.L)};
+    if (!encode(&p.tm_u, p.u, bf16, 2, dims_u, pitch2, box2) ||
         !encode(&p.tm_dl, p.delta, bf16, 2, dims_kbl, pitch2, box2) ||
         (need_z && !encode(&p.tm_z, p.z, bf16, 2, dims_bl, pitch2, box2)))
         return cudaErrorInvalidValue;
@@ -1036,7 +1039,9 @@ cudaError_t make_maps(ScanParams& p, bool need_z)
         const cuuint64_t pitch3[2] = {D * esz, static_cast<cuuint64_t>(p.W) * D * esz};
         const cuuint64_t dims3[3] = {D, static_cast<cuuint64_t>(p.W),
                                      static_cast<cuuint64_t>(p.batch * p.H)};
-        if (!encode(&p.tm_u3, p.u, bf16, 3, dims3, pitch3, box3) ||
+        const cuuint64_t dims3u[3] = {D, static_cast<cuuint64_t>(p.W),
+                                      static_cast<cuuint64_t>(u_blocks * p.H)};
+        if (!encode(&p.tm_u3, p.u, bf16, 3, dims3u, pitch3, box3) ||
             (need_z && !encode(&p.tm_z3, p.z, bf16, 3, dims3, pitch3, box3)))
             return cudaErrorInvalidValue;
     }

@@ -25,6 +25,7 @@ SS_DIR_FWD, SS_DIR_REV, SS_DIR_COL, SS_DIR_COL_REV = 0, 1, 2, 3
 SS_FLAG_GENERIC_A = 1
 SS_FLAG_ZOH_EXACT = 2
 SS_FLAG_TEST_WAIT_TIMEOUT = 8
+SS_FLAG_U_PER_DIRECTION = 16
 SS_ERR_DEVICE_TIMEOUT = 9
 SS_MAX_DSTATE = 16
 SS_MAX_DIRS = 4
@@ -279,7 +280,8 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
                        conv_weight=None, conv_bias=None):
     """Selective scan forward on CUDA tensors.
 
-    u, z: [batch, L, D]; delta: [K, batch, L, D] (or [batch, L, D] when K = 1); B, C:
+    u, z: [batch, L, D] (u may be [K, batch, L, D]: direction k scans its own input u[k],
+    e.g. the two modalities of a cross-modal scan); delta: [K, batch, L, D] (or [batch, L, D] when K = 1); B, C:
     [K, batch, L, N] (or [batch, L, N]); A: [D, N] float32; D (skip) and delta_bias: [D] float32.
     u, delta, B, C, z share one dtype (float32 or bfloat16); out has that dtype.
     initial_state: [K, batch, D, N] float32 state before step 0 (None = zero); zoh_exact: use
@@ -291,10 +293,12 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     """
     import torch
     device = u.device
-    if u.dim() != 3:
-        raise ValueError("u must be [batch, L, D]")
-    batch, L, Dm = u.shape
     K = len(dirs)
+    if u.dim() == 4 and u.shape[0] == K:
+        flags = int(flags) | SS_FLAG_U_PER_DIRECTION
+    elif u.dim() != 3:
+        raise ValueError("u must be [batch, L, D] or [K, batch, L, D]")
+    batch, L, Dm = u.shape[-3:]
     if delta.dim() == 3:
         delta = delta.unsqueeze(0)
     if B.dim() == 3:
@@ -304,7 +308,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     N = A.shape[-1]
     io = u.dtype
     _io_code(io)
-    _check(u, "u", (batch, L, Dm), io, device)
+    _check(u, "u", tuple(u.shape[:-3]) + (batch, L, Dm), io, device)
     _check(delta, "delta", (K, batch, L, Dm), io, device)
     _check(B, "B", (K, batch, L, N), io, device)
     _check(C, "C", (K, batch, L, N), io, device)
@@ -313,7 +317,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     _check(D, "D", (Dm,), torch.float32, device)
     _check(delta_bias, "delta_bias", (Dm,), torch.float32, device)
     if out is None:
-        out = torch.empty_like(u)
+        out = torch.empty((batch, L, Dm), dtype=io, device=device)
     _check(out, "out", (batch, L, Dm), io, device)
     if return_last_state and last_state is None:
         last_state = torch.empty((K, batch, Dm, N), dtype=torch.float32, device=device)

@@ -121,6 +121,12 @@ def test_null_alignment_and_workspace_errors():
         scan.selective_scan_workspace_size(sh, None, o)
 
 
+def test_input_per_direction_flag_accepted():
+    sh = _shape()
+    o = scan.make_opts(flags=scan.SS_FLAG_U_PER_DIRECTION)
+    assert scan.selective_scan_workspace_size(sh, scan.make_dirmap((0, 0)), o) > 0
+
+
 def test_conv_options_validated():
     sh = _shape()
     ok = scan.make_opts(conv_weight=FAKE, conv_bias=FAKE, conv_width=4)

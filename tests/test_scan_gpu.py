@@ -240,6 +240,29 @@ def test_conv_with_initial_state_and_exact_zoh(cuda_device):
     _check(inp, cuda_device, segments=2, initial_state=h0, zoh_exact=True)
 
 
+# ----------------------------------------------------------------------------- input per direction
+
+@pytest.mark.parametrize("segments", [0, 3])
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F32])
+def test_cromb_cross_modal(cuda_device, dtype, segments):
+    w = wl.variant("cromb", name="cromb_small", batch=2, seqlen=333, dim=72, dtype=dtype, seed=140)
+    _check(wl.make_inputs(w), cuda_device, segments=segments)
+
+
+def test_input_per_direction_all_orders_with_conv_and_gate(cuda_device):
+    w = wl.Workload("upd", 2, 16 * 6, 64, 16, wl.BF16, dirs=(wl.DIR_FORWARD, wl.DIR_COLUMN,
+                                                           wl.DIR_REVERSE, wl.DIR_COLUMN_REVERSE),
+                    H=16, W=6, u_per_dir=True, conv=4, seed=141)
+    _check(wl.make_inputs(w), cuda_device, segments=2)
+
+
+def test_input_per_direction_row_by_row_columns(cuda_device):
+    # H % 8 != 0: column orders copy u row by row, from direction k's own input
+    w = wl.Workload("upd2", 2, 10 * 7, 32, 8, wl.F32, dirs=(wl.DIR_COLUMN_REVERSE, wl.DIR_FORWARD),
+                    H=10, W=7, u_per_dir=True, seed=142)
+    _check(wl.make_inputs(w), cuda_device)
+
+
 # ----------------------------------------------------------------------------- full size
 
 FULL_SAMPLES = {
@@ -250,10 +273,11 @@ FULL_SAMPLES = {
     "vim": (8, 32),
     "ss2d": (4, 16),
     "m130_conv": (None, 24),
+    "cromb": (4, 16),
 }
 
 
-@pytest.mark.parametrize("name", ["tiny", "m130", "long", "vim", "ss2d", "m130_conv"])
+@pytest.mark.parametrize("name", ["tiny", "m130", "long", "vim", "ss2d", "m130_conv", "cromb"])
 def test_full_size_workloads_sampled(cuda_device, name):
     import torch
     w = wl.variant("m130", conv=4) if name == "m130_conv" else wl.WORKLOADS[name]
