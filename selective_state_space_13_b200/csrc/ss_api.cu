@@ -272,6 +272,9 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
     p.zoh = (pl.flags & SS_FLAG_ZOH_EXACT) ? 1 : 0;
     p.test_timeout = (pl.flags & SS_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
     p.u_per_dir = (pl.flags & SS_FLAG_U_PER_DIRECTION) ? 1 : 0;
+    p.status = ss::status_word();
+    if (!p.status)
+        return SS_ERR_CUDA;
     p.init_state = pl.init_state;
     p.conv_w = pl.conv_w;
     p.conv_b = pl.conv_b;

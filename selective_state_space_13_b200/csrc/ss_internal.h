@@ -50,6 +50,7 @@ struct ScanParams {
     int32_t test_timeout;   // 1: test hook, wait on a barrier nothing completes and report
     int32_t conv_width;     // taps of conv_w (1..SS_MAX_CONV_WIDTH) when conv_w is set
     int32_t u_per_dir;      // 1: direction k reads its own input u[k]
+    unsigned int* status;   // the device error word (status_word()), or'ed by bounded waits
 };
 
 struct MergeParams {
@@ -63,6 +64,14 @@ struct MergeParams {
 
 // Channels handled by one CTA of the scan kernel (one thread per channel).
 int channels_per_cta();
+
+// Device address of the library's error word on the current device (looked up once per device),
+// or null if the runtime fails.
+unsigned int* status_word();
+
+// The scan launches of one io type (one translation unit each).
+cudaError_t launch_scan_f32(const ScanParams& p, int phase1, cudaStream_t stream);
+cudaError_t launch_scan_bf16(const ScanParams& p, int phase1, cudaStream_t stream);
 
 // Enqueue one scan launch.  phase1 = 1: segment aggregates only (segments 0..S-2);
 // phase1 = 0: full scan of all S segments.  Returns the CUDA error of the launch.
