@@ -19,6 +19,8 @@ Readings of the pages that the oracle fixes (each is listed with its reason in t
     as the same gate.
   * With several directions every direction adds its own Dskip*u (each is a full S6 scan).
   * The state starts at zero unless an initial state is given.
+  * Delta may arrive as int8 codes q with one scale per channel: the raw value is q * scale[d]
+    ("S4 -> Mamba" sec. 2.3; the pages give no scale convention).
   * With u given per direction ([K, batch, L, D]), direction k scans its own input; Sigma's
     CroMB ("S4 -> Mamba" sec. 4.1) is two such directions in forward order with the C of the
     other modality, summed.
@@ -67,7 +69,7 @@ def _load():
             lib.ss_oracle_scan.restype = ctypes.c_int
             lib.ss_oracle_scan.argtypes = [i64, i64, i64, i64, i32, dp, i64, i64,
                                            dp, dp, dp, dp, dp, dp, dp, dp,
-                                           i32, i32, dp, dp, i32, dp, dp, dp, i64, i32]
+                                           i32, i32, dp, dp, i32, dp, dp, dp, i64, i32, dp]
             lib.ss_oracle_conv_silu.restype = ctypes.c_int
             lib.ss_oracle_conv_silu.argtypes = [i64, i64, i64, i32, dp, i64, i64, dp, dp, dp,
                                                 i64, dp]
@@ -122,13 +124,15 @@ def conv_silu(u, conv_weight, conv_bias=None, dirs=(DIR_FORWARD,), H=0, W=0):
 def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softplus=True,
                    dirs=(DIR_FORWARD,), H=0, W=0, zoh_exact=False, threads=None,
                    return_last_state=True, initial_state=None, conv_weight=None,
-                   conv_bias=None):
+                   conv_bias=None, delta_scale=None):
     """Run the oracle.
 
     u, z: [batch, L, D] (u may be [K, batch, L, D]: direction k then reads u[k], as in the
     cross-modal scan); delta: [K, batch, L, D]; B, C: [K, batch, L, N]; A: [D, N];
     Dskip, delta_bias: [D] or None; initial_state: [K, batch, D, N] or None (zero);
-    conv_weight: [K, D, width] or None (u is used as it is); conv_bias: [K, D] or None.
+    conv_weight: [K, D, width] or None (u is used as it is); conv_bias: [K, D] or None;
+    delta_scale: [D] or None -- with it, delta holds int8 codes q and the raw value is
+    q * delta_scale[d].
     Inputs may be any real dtype; they are upcast to float64 exactly.  Returns
     (out [batch, L, D], last_state [K, batch, D, N]) in float64.
     """
@@ -136,6 +140,7 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
     Dskip, z, delta_bias = _f64(Dskip), _f64(z), _f64(delta_bias)
     initial_state = _f64(initial_state)
     conv_weight, conv_bias = _f64(conv_weight), _f64(conv_bias)
+    delta_scale = _f64(delta_scale)
     dirs_arr = np.ascontiguousarray(np.asarray(dirs, dtype=np.int32).reshape(-1))
     K = int(dirs_arr.size)
     u_per_dir = u.ndim == 4
@@ -151,9 +156,9 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
         raise ValueError("B and C must be [K, batch, L, N]")
     if z is not None and z.shape != (batch, L, D):
         raise ValueError("z must be [batch, L, D]")
-    for v in (Dskip, delta_bias):
+    for v in (Dskip, delta_bias, delta_scale):
         if v is not None and v.shape != (D,):
-            raise ValueError("Dskip and delta_bias must be [D]")
+            raise ValueError("Dskip, delta_bias and delta_scale must be [D]")
     if initial_state is not None and initial_state.shape != (K, batch, D, N):
         raise ValueError("initial_state must be [K, batch, D, N]")
     if conv_weight is not None:
@@ -170,7 +175,7 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
                                 int(bool(zoh_exact)), _ptr(out), _ptr(last), int(threads),
                                 _ptr(initial_state), _ptr(conv_weight), _ptr(conv_bias),
                                 0 if conv_weight is None else int(conv_weight.shape[2]),
-                                int(u_per_dir))
+                                int(u_per_dir), _ptr(delta_scale))
     if rc != 0:
         raise ValueError("oracle rejected its arguments (code %d)" % rc)
     return out, last

@@ -24,6 +24,8 @@
  *       Delta = softplus(delta[k,b,t,d] + bias[d])         ("Understanding Mamba from zero",
  *               (or the raw sum when softplus is off)       sec. 4.1 Algorithm 2 / sec. 6.2
  *                                                          Step 3: tau_Delta(Parameter+s_Delta))
+ *               with int8 codes (delta_scale given), the   ("S4 -> Mamba" sec. 2.3: Delta
+ *               raw value is delta[k,b,t,d] * delta_scale[d] quantised to int8 at inference)
  *       for n: Abar = exp(Delta * A[d,n])                  (same page, sec. 6.2 Step 4, eq. 4)
  *              Bbar = Delta * B[k,b,t,n]                   (first-order reading of eq. 4, as on
  *                                                          "Mamba-UNet" sec. 4: Bbar ~ Delta*B)
@@ -63,6 +65,7 @@
  *   initial_state        [K, batch, D, N] or NULL (zero)
  *   conv_weight          [K, D, conv_width] or NULL (no convolution: u_t = u[b,p,d])
  *   conv_bias            [K, D] or NULL (zero)
+ *   delta_scale          [D] or NULL: delta holds int8 codes q, the raw value is q * scale[d]
  *
  * Parity is pinned by tests/test_oracle_pins.py against the LTI convolution form (eq. 3),
  * Theorem 1, the unrolled double sum, the Delta -> 0 limit, reversal and explicitly permuted
@@ -164,7 +167,8 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                    int32_t softplus, int32_t zoh_exact,
                    double* out, double* last_state, int32_t nthreads,
                    const double* initial_state, const double* conv_weight,
-                   const double* conv_bias, int64_t conv_width, int32_t u_per_direction)
+                   const double* conv_bias, int64_t conv_width, int32_t u_per_direction,
+                   const double* delta_scale)
 {
     int bad = 0;
     if (batch < 0 || L < 0 || D < 0 || N < 1 || K < 1 || K > 4)
@@ -220,7 +224,9 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                                       conv_bias ? conv_bias[(int64_t)k * D + d] : 0.0, conv_width)
                                 : uk[(b * L + p) * D + d];
                         const int64_t row = ((int64_t)k * batch + b) * L + t;
-                        double dt = delta[row * D + d] + (delta_bias ? delta_bias[d] : 0.0);
+                        const double draw = delta_scale ? delta[row * D + d] * delta_scale[d]
+                                                        : delta[row * D + d];
+                        double dt = draw + (delta_bias ? delta_bias[d] : 0.0);
                         if (softplus)
                             dt = oracle_softplus(dt);
                         double yt = 0.0;

@@ -15,6 +15,10 @@ Recipe (identical for every workload, seed = 20260 + workload index):
   * Dskip = 1 (fp32), except the tiny workload where Dskip ~ N(0, 1);
   * delta_bias: Delta0 ~ exp(U[ln 1e-3, ln 0.1]) per channel, bias = softplus^-1(Delta0) =
     Delta0 + log(-expm1(-Delta0)); the tiny workload uses bias = 0;
+  * with int8 Delta (`delta_int8`): delta_raw is drawn as above in float32, then quantised
+    symmetrically per channel: scale[d] = max |delta_raw[:, :, :, d]| / 127 over directions,
+    batch rows and steps, q = round-half-even(delta_raw / scale[d]) (in [-127, 127]); the
+    arrays are the int8 codes and the float32 scales;
   * with a causal convolution of `conv` taps before the scan (no named workload has one; the
     variants that test it do): taps and bias per direction and channel ~ U(-1/sqrt(conv),
     1/sqrt(conv)) in fp32, the usual initial scale of a depthwise convolution of that width
@@ -59,6 +63,7 @@ class Workload:
     seed: int = 20260
     conv: int = 0                   # taps of the causal convolution before the scan (0: none)
     u_per_dir: bool = False         # one input u[k] per direction ([K, batch, L, D])
+    delta_int8: bool = False        # delta_raw as int8 codes with one fp32 scale per channel
     extra: dict = field(default_factory=dict, compare=False)
 
     @property
@@ -81,7 +86,9 @@ class Workload:
         bln = self.batch * self.seqlen * self.dstate
         nbytes = bld * e * ((self.K if self.u_per_dir else 1) + 1 + (1 if self.gate else 0))
         # u (per direction or shared), out, z
-        nbytes += self.K * bld * e                                 # delta_raw per direction
+        nbytes += self.K * bld * (1 if self.delta_int8 else e)     # delta_raw per direction
+        if self.delta_int8:
+            nbytes += self.dim * 4                                 # its scales
         nbytes += 2 * self.K * bln * e                             # B, C per direction
         nbytes += self.dim * self.dstate * 4 + 2 * self.dim * 4    # A, Dskip, delta_bias
         if with_last_state:
@@ -192,8 +199,12 @@ def make_inputs(w: Workload | str, threads: int | None = None) -> dict:
     else:
         u = _normal((b, L, D), ss(0), w.dtype, threads)
     z = _normal((b, L, D), ss(1), w.dtype, threads) if w.gate else None
-    delta = np.stack([_normal((b, L, D), ss(2, k), w.dtype, threads) for k in range(K)]) \
-        if K > 1 else _normal((b, L, D), ss(2, 0), w.dtype, threads)[None]
+    ddtype = F32 if w.delta_int8 else w.dtype
+    delta = np.stack([_normal((b, L, D), ss(2, k), ddtype, threads) for k in range(K)]) \
+        if K > 1 else _normal((b, L, D), ss(2, 0), ddtype, threads)[None]
+    delta_scale = None
+    if w.delta_int8:
+        delta, delta_scale = quantize_int8_per_channel(delta)
     B = np.stack([_normal((b, L, N), ss(3, k), w.dtype, threads) for k in range(K)])
     C = np.stack([_normal((b, L, N), ss(4, k), w.dtype, threads) for k in range(K)])
     g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([root, 5])))
@@ -214,7 +225,17 @@ def make_inputs(w: Workload | str, threads: int | None = None) -> dict:
         conv_weight = gc.uniform(-lim, lim, size=(K, D, w.conv)).astype(np.float32)
         conv_bias = gc.uniform(-lim, lim, size=(K, D)).astype(np.float32)
     return dict(workload=w, u=u, z=z, delta=delta, B=B, C=C, A=A, Dskip=Dskip, delta_bias=bias,
-                conv_weight=conv_weight, conv_bias=conv_bias)
+                conv_weight=conv_weight, conv_bias=conv_bias, delta_scale=delta_scale)
+
+
+def quantize_int8_per_channel(x: np.ndarray):
+    """Symmetric int8 codes of a float32 [..., D] array with one scale per channel (the last
+    axis): scale = max |x| / 127 over all other axes, codes = round-half-even(x / scale)."""
+    D = x.shape[-1]
+    amax = np.abs(x.reshape(-1, D)).max(axis=0).astype(np.float32)
+    scale = np.where(amax > 0, amax / np.float32(127.0), np.float32(1.0)).astype(np.float32)
+    q = np.rint(x / scale).clip(-127, 127).astype(np.int8)
+    return q, scale
 
 
 def inputs_f64(inp: dict, channels=None, batches=None) -> dict:
@@ -228,6 +249,8 @@ def inputs_f64(inp: dict, channels=None, batches=None) -> dict:
             return None
         v = x[:, bsel] if lead else x[bsel]
         v = v[..., dsel]
+        if v.dtype == np.int8:
+            return v.astype(np.float64)
         return to_f64(v, w.dtype)
 
     def bc(x):
@@ -243,6 +266,8 @@ def inputs_f64(inp: dict, channels=None, batches=None) -> dict:
                 np.asarray(inp["conv_weight"][:, dsel], dtype=np.float64),
                 conv_bias=None if inp.get("conv_bias") is None else
                 np.asarray(inp["conv_bias"][:, dsel], dtype=np.float64),
+                delta_scale=None if inp.get("delta_scale") is None else
+                np.asarray(inp["delta_scale"][dsel], dtype=np.float64),
                 softplus=w.softplus, dirs=w.dirs, H=w.H, W=w.W)
 
 
@@ -266,4 +291,5 @@ def to_device(inp: dict, device) -> dict:
                 D=to_torch(inp["Dskip"], F32, device),
                 delta_bias=to_torch(inp["delta_bias"], F32, device),
                 conv_weight=to_torch(inp.get("conv_weight"), F32, device),
-                conv_bias=to_torch(inp.get("conv_bias"), F32, device))
+                conv_bias=to_torch(inp.get("conv_bias"), F32, device),
+                delta_scale=to_torch(inp.get("delta_scale"), F32, device))

@@ -50,7 +50,8 @@ def run_gpu(inp, dev_inputs=None, device="cuda:0", segments=0, flags=0, use_z=Tr
         softplus=w.softplus if softplus is None else softplus, dirs=w.dirs, H=w.H, W=w.W,
         return_last_state=True, segments=segments, flags=flags, initial_state=h0,
         zoh_exact=zoh_exact, conv_weight=t.get("conv_weight"),
-        conv_bias=t.get("conv_bias") if use_conv_bias else None)
+        conv_bias=t.get("conv_bias") if use_conv_bias else None,
+        delta_scale=t.get("delta_scale"))
     return out, last
 
 
@@ -65,4 +66,5 @@ def run_oracle(inp, channels=None, batches=None, use_z=True, use_D=True, use_bia
                                  softplus=w.softplus if softplus is None else softplus,
                                  dirs=w.dirs, H=w.H, W=w.W, initial_state=initial_state,
                                  zoh_exact=zoh_exact, conv_weight=f["conv_weight"],
-                                 conv_bias=f["conv_bias"] if use_conv_bias else None)
+                                 conv_bias=f["conv_bias"] if use_conv_bias else None,
+                                 delta_scale=f["delta_scale"])

@@ -53,6 +53,11 @@ MUTATIONS = [
      "                                      conv_weight + ((int64_t)k * D + d) * conv_width,",
      "uk, b, d, L, D, dirs[k], H, W, t,\n"
      "                                      conv_weight + ((int64_t)0 * D + d) * conv_width,"),
+    ("int8 scale of the first channel", "delta[row * D + d] * delta_scale[d]",
+     "delta[row * D + d] * delta_scale[0]"),
+    ("int8 scale applied after the bias", "double dt = draw + (delta_bias ? delta_bias[d] : 0.0);",
+     "double dt = (delta_scale ? (delta[row * D + d] + (delta_bias ? delta_bias[d] : 0.0)) * "
+     "delta_scale[d] : draw + (delta_bias ? delta_bias[d] : 0.0));"),
     ("every direction reads the first input", "u_per_direction ? u + (int64_t)k * batch",
      "u_per_direction ? u + (int64_t)0 * batch"),
 ]

@@ -35,6 +35,8 @@ identity, a special case or a brute force that does not run the oracle's recurre
       scans of those inputs, gated; and Sigma's CroMB ("S4 -> Mamba" sec. 4.1) written as the
       pages give it, SSM(x_rgb, C=C_depth) + SSM(x_depth, C=C_rgb) from two separate scans,
       equals the two-direction scan with the C tensors stacked in swapped order.
+  P12 int8 Delta ("S4 -> Mamba" sec. 2.3): codes q with one scale per channel scan exactly like
+      the raw values q * scale[d] given directly (the products are exact in float64).
   plus the silu gate against sigmoid written out, a hand-worked Abar = 1/2 example, empty and
   length-1 inputs, and a regression fixture written by tests/golden/make_golden.py.
 """
@@ -548,3 +550,24 @@ def test_P11_cromb_cross_modal_scan():
                                    np.concatenate([B_rgb, B_depth]),
                                    np.concatenate([C_depth, C_rgb]), dirs=(FWD, FWD), **args)
     assert rel_err(out, out_rgb + out_depth) < 1e-13
+
+
+# ----------------------------------------------------------------------------- P12 (int8 Delta)
+
+@pytest.mark.parametrize("softplus", [True, False])
+def test_P12_int8_delta_codes_with_channel_scales(softplus):
+    rng = np.random.default_rng(95)
+    batch, L, D, N, K = 2, 27, 5, 4, 2
+    c = rand_case(rng, batch, L, D, N, K=K)
+    q = rng.integers(-127, 128, size=(K, batch, L, D)).astype(np.float64)
+    scale = rng.uniform(0.002, 0.05, size=D).astype(np.float32).astype(np.float64)
+    args = dict(Dskip=c["Dskip"], delta_bias=c["delta_bias"], softplus=softplus, z=c["z"],
+                dirs=(FWD, REV))
+    out, last = oracle.selective_scan(c["u"], q, c["A"], c["B"], c["C"], delta_scale=scale, **args)
+    raw = q * scale[None, None, None, :]              # exact: 8-bit codes times 24-bit scales
+    ref, ref_last = oracle.selective_scan(c["u"], raw, c["A"], c["B"], c["C"], **args)
+    assert np.array_equal(out, ref) and np.array_equal(last, ref_last)
+    # and a scale is not an offset: scaling the codes by 2 and halving the scale is the same scan
+    out2, _ = oracle.selective_scan(c["u"], 2 * q, c["A"], c["B"], c["C"], delta_scale=scale / 2,
+                                    **args)
+    assert np.array_equal(out2, out)
