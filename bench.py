@@ -171,8 +171,8 @@ def workload_of(args) -> wl.Workload:
         if w.H:
             raise SystemExit("--seqlen does not apply to image workloads")
         w = wl.variant(w.name, seqlen=args.seqlen)
-    if args.conv:
-        w = wl.variant(w.name, seqlen=w.seqlen, conv=args.conv)
+    if args.conv or args.delta_int8:
+        w = wl.variant(w.name, seqlen=w.seqlen, conv=args.conv, delta_int8=args.delta_int8)
     return w
 
 
@@ -180,6 +180,8 @@ def describe(w: wl.Workload) -> str:
     text = wl.DESCRIPTIONS[w.name]
     if w.conv:
         text += ", causal depthwise conv1d (%d taps) + SiLU fused before the scan" % w.conv
+    if w.delta_int8:
+        text += ", int8 Delta codes with per-channel scales"
     return text
 
 
@@ -205,7 +207,7 @@ def time_oracle(inp, channels, threads):
     oracle.selective_scan(f["u"], f["delta"], f["A"], f["B"], f["C"], Dskip=f["Dskip"], z=f["z"],
                           delta_bias=f["delta_bias"], softplus=w.softplus, dirs=w.dirs, H=w.H,
                           W=w.W, threads=threads, conv_weight=f["conv_weight"],
-                          conv_bias=f["conv_bias"])
+                          conv_bias=f["conv_bias"], delta_scale=f["delta_scale"])
     return time.perf_counter() - t0
 
 
@@ -238,7 +240,8 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded, %s)" % describe(w),
-            "config": {"workload": describe(w), "name": w.name, "conv": w.conv},
+            "config": {"workload": describe(w), "name": w.name, "conv": w.conv,
+                       "delta_int8": w.delta_int8},
             "updates_per_s": w.updates() * frac / step_s,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": sample},
@@ -277,7 +280,7 @@ def run_ours(args):
                                 delta_bias=t["delta_bias"], softplus=w.softplus, dirs=w.dirs,
                                 H=w.H, W=w.W, out=out, last_state=last, segments=args.segments,
                                 flags=args.flags, events=events, conv_weight=t["conv_weight"],
-                                conv_bias=t["conv_bias"])
+                                conv_bias=t["conv_bias"], delta_scale=t["delta_scale"])
 
     # plan facts for the report
     shape = scan.make_shape(w.batch, w.seqlen, w.dim, w.dstate,
@@ -392,7 +395,7 @@ def run_ours(args):
                                                    w.updates() * frac)}
 
     traffic = None if args.seqlen else recorded_traffic(
-        w.name + ("_conv%d" % w.conv if w.conv else ""))
+        w.name + ("_conv%d" % w.conv if w.conv else "") + ("_int8" if w.delta_int8 else ""))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
@@ -404,6 +407,7 @@ def run_ours(args):
                    "name": w.name, "batch": w.batch,
                    "seqlen": w.seqlen, "dim": w.dim, "dstate": w.dstate, "directions": w.K,
                    "gate": w.gate, "returns_last_state": want_last, "conv": w.conv,
+                   "delta_int8": w.delta_int8,
                    "parallelism": "independent problems per rank" if world > 1 else "1 GPU",
                    "l2": "flushed (256 MiB write) before every timed step",
                    "segments": args.segments or "auto", "workspace_bytes": ws_bytes},
@@ -448,6 +452,8 @@ def parse(argv=None):
                     help="override the workload's sequence length (smaller cases for profiling)")
     ap.add_argument("--conv", type=int, default=0,
                     help="taps of a causal depthwise conv1d + SiLU fused before the scan (0 = none)")
+    ap.add_argument("--delta-int8", action="store_true",
+                    help="Delta as int8 codes with one scale per channel")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-updates", type=float, default=4e9,

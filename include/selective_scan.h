@@ -12,7 +12,9 @@
  *              before step 0                                Mamba" sec. 2.2
  *   Delta_t  = softplus(delta_raw_t + delta_bias)          "Understanding Mamba from zero",
  *                                                           sec. 4.1 Algorithm 2 and sec. 6.2
- *                                                           Step 3 (tau_Delta(Parameter+s_Delta))
+ *                                                           Step 3 (tau_Delta(Parameter+s_Delta));
+ *              delta_raw may arrive as int8 codes times     int8 Delta at inference, "S4 ->
+ *              one scale per channel (SS_FLAG_DELTA_INT8)   Mamba" sec. 2.3
  *   Abar_t   = exp(Delta_t * A)                            same page, sec. 6.2 Step 4, eq. (4)
  *   Bbar_t u = Delta_t * B_t * u_t                         first-order form of eq. (4), as
  *                                                           "Mamba-UNet" sec. 4 writes it
@@ -52,7 +54,7 @@
 extern "C" {
 #endif
 
-#define SS_ABI_VERSION 3
+#define SS_ABI_VERSION 4
 #define SS_MAX_DSTATE 16
 #define SS_MAX_DIRS 4
 #define SS_MAX_CONV_WIDTH 4
@@ -119,6 +121,8 @@ typedef struct {
                                 conv_weight)                                                 */
     int32_t conv_width;      /* taps, 1..SS_MAX_CONV_WIDTH with conv_weight; 0 without      */
     int32_t reserved;        /* must be 0                                                    */
+    const float* delta_scale; /* [D] fp32 device array with SS_FLAG_DELTA_INT8 (delta_raw =
+                                 code * delta_scale[d]); NULL otherwise                      */
 } ss_launch_opts;
 
 #define SS_FLAG_GENERIC_A 1 /* never use the exp-power shortcut for A[d,n] = (n+1)*A[d,0]   */
@@ -131,6 +135,11 @@ typedef struct {
                                       Mamba" sec. 4.1) is two forward directions over the two
                                       modalities' inputs with the C tensors stacked in swapped
                                       order, so that each modality reads the other's C      */
+#define SS_FLAG_DELTA_INT8 32 /* delta holds int8 codes [K, batch, L, D] (one byte each); the
+                                 raw value is code * delta_scale[d] (ss_launch_opts).  Needs
+                                 io_dtype SS_BF16 and dim a multiple of 16 (the code rows are
+                                 dim bytes; SS_ERR_ALIGN otherwise); the base pointer follows
+                                 the 16-byte rule                                        */
 #define SS_FLAG_TEST_WAIT_TIMEOUT 8 /* test hook for failure detection: every CTA waits (20 ms
                                        at most) on a barrier that nothing completes, gives up,
                                        records SS_ERR_DEVICE_TIMEOUT for
@@ -149,7 +158,8 @@ ss_status selective_scan_workspace_size(const ss_shape* shape, const ss_directio
  *   shape       problem sizes and io dtype (host pointer)
  *   u           [batch, L, D]      io dtype, spatial order ([K, batch, L, D] with
  *                                  SS_FLAG_U_PER_DIRECTION)
- *   delta       [K, batch, L, D]   io dtype, raw Delta of direction k in its scan order
+ *   delta       [K, batch, L, D]   io dtype (int8 codes with SS_FLAG_DELTA_INT8), raw Delta of
+ *                                  direction k in its scan order
  *   A           [D, N]             fp32, shared by all directions
  *   B, C        [K, batch, L, N]   io dtype, scan order of direction k
  *   Dskip       [D] fp32, or NULL for zero

@@ -35,6 +35,7 @@ struct Plan {
     const float* conv_w;
     const float* conv_b;
     int conv_width;
+    const float* delta_scale;
     // workspace layout (byte offsets, 0 size = unused)
     size_t off_carry_h, off_carry_s, off_ypart, bytes;
 };
@@ -106,6 +107,7 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
     pl->init_state = nullptr;
     pl->conv_w = pl->conv_b = nullptr;
     pl->conv_width = 0;
+    pl->delta_scale = nullptr;
     if (opts) {
         if (opts->reserved != 0)
             return SS_ERR_UNSUPPORTED;
@@ -121,8 +123,19 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
         if (opts->segments < 0 || opts->segments > kMaxSegments)
             return SS_ERR_UNSUPPORTED;
         if (opts->flags & ~(SS_FLAG_GENERIC_A | SS_FLAG_ZOH_EXACT | SS_FLAG_TEST_WAIT_TIMEOUT |
-                            SS_FLAG_U_PER_DIRECTION))
+                            SS_FLAG_U_PER_DIRECTION | SS_FLAG_DELTA_INT8))
             return SS_ERR_UNSUPPORTED;
+        if (opts->flags & SS_FLAG_DELTA_INT8) {
+            if (s->io_dtype != SS_BF16)
+                return SS_ERR_UNSUPPORTED;
+            if (!opts->delta_scale)
+                return SS_ERR_NULL;
+            if (s->dim % 16 != 0)
+                return SS_ERR_ALIGN;
+            pl->delta_scale = opts->delta_scale;
+        } else if (opts->delta_scale) {
+            return SS_ERR_UNSUPPORTED;
+        }
         pl->init_state = opts->initial_state;
         seg = opts->segments;
         pl->flags = opts->flags;
@@ -219,7 +232,8 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
     for (const void* p : {static_cast<const void*>(A), static_cast<const void*>(Dskip),
                           static_cast<const void*>(delta_bias), static_cast<const void*>(last_state),
                           static_cast<const void*>(pl.init_state),
-                          static_cast<const void*>(pl.conv_w), static_cast<const void*>(pl.conv_b)})
+                          static_cast<const void*>(pl.conv_w), static_cast<const void*>(pl.conv_b),
+                          static_cast<const void*>(pl.delta_scale)})
         if (p && !aligned(p, 4))
             return SS_ERR_ALIGN;
     if (pl.bytes > 0 && (!workspace || workspace_bytes < pl.bytes))
@@ -279,6 +293,7 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
     p.conv_w = pl.conv_w;
     p.conv_b = pl.conv_b;
     p.conv_width = pl.conv_width;
+    p.delta_scale = pl.delta_scale;
 
     // the timing events bracket the scan pipeline: the segment-aggregate launch (if any) and
     // the scan launch, which may overlap (nothing is recorded between them)

@@ -23,7 +23,7 @@ struct ScanParams {
     CUtensorMap tm_dl;         // delta as [K*batch*L rows, D], same boxes
     CUtensorMap tm_u3, tm_z3;  // u, z as [batch*H, W, D]: boxes of 8 image rows of one column
     const void* u;          // [batch, L, D] io, spatial order ([K, batch, L, D] with u_per_dir)
-    const void* delta;      // [K, batch, L, D] io, scan order
+    const void* delta;      // [K, batch, L, D] io (or int8 codes), scan order
     const float* A;         // [D, N]
     const void* B;          // [K, batch, L, N] io, scan order
     const void* C;          // [K, batch, L, N] io, scan order
@@ -36,6 +36,7 @@ struct ScanParams {
     const float* init_state;  // [K, batch, D, N] state before step 0, or null (zero)
     const float* conv_w;    // [K, D, conv_width] causal conv taps per direction, or null
     const float* conv_b;    // [K, D] conv bias, or null (zero)
+    const float* delta_scale;  // [D] scale of int8 delta codes, or null (delta in io type)
     float* carry_h;         // [K, batch, S, D, N] end state of each segment scanned from zero
     float* carry_s;         // [K, batch, S, D] sum over the segment of Delta*log2(e)
     int64_t batch, L, D;
@@ -72,6 +73,7 @@ unsigned int* status_word();
 // The scan launches of one io type (one translation unit each).
 cudaError_t launch_scan_f32(const ScanParams& p, int phase1, cudaStream_t stream);
 cudaError_t launch_scan_bf16(const ScanParams& p, int phase1, cudaStream_t stream);
+cudaError_t launch_scan_bf16_i8(const ScanParams& p, int phase1, cudaStream_t stream);
 
 // Enqueue one scan launch.  phase1 = 1: segment aggregates only (segments 0..S-2);
 // phase1 = 0: full scan of all S segments.  Returns the CUDA error of the launch.

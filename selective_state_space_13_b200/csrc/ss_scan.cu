@@ -36,6 +36,8 @@ int channels_per_cta() { return 32 * kWarps; }
 
 cudaError_t launch_scan(const ScanParams& p, int io_dtype, int phase1, cudaStream_t stream)
 {
+    if (p.delta_scale)
+        return launch_scan_bf16_i8(p, phase1, stream);  // int8 delta needs bf16 io
     return io_dtype == SS_BF16 ? launch_scan_bf16(p, phase1, stream)
                                : launch_scan_f32(p, phase1, stream);
 }

@@ -234,6 +234,9 @@ __device__ __forceinline__ float expm1_acc(float x)
 // ---------------------------------------------------------------------------- element types
 
 template <typename T> struct Io;
+template <> struct Io<int8_t> {  // int8 Delta codes (loaded only)
+    static __device__ __forceinline__ float ld(const int8_t* p) { return static_cast<float>(*p); }
+};
 template <> struct Io<float> {
     static __device__ __forceinline__ float ld(const float* p) { return *p; }
     static __device__ __forceinline__ float st(float v) { return v; }
@@ -268,11 +271,12 @@ __host__ __device__ __forceinline__ int64_t position(int32_t dir, int64_t L, int
 
 // One pipeline stage holds kTile rows of u, delta and z for the CTA's channels (as copied),
 // the raw B and C tiles, their fp32 copies, and the output row offsets of the tile.
-template <typename io_t, int NS, int WARPS, bool GATE, bool PHASE1, int STAGES>
+template <typename io_t, typename dl_t, int NS, int WARPS, bool GATE, bool PHASE1, int STAGES>
 struct Layout {
     static constexpr int DC = 32 * WARPS;                           // channels per CTA
     static constexpr int ROW = DC * (int)sizeof(io_t);               // bytes of one row slice
     static constexpr int ROWS = kTile * ROW;                         // bytes of one tensor tile
+    static constexpr int ROWS_DL = kTile * DC * (int)sizeof(dl_t);   // bytes of one delta tile
     static constexpr int BCRAW = ((kTile * NS * (int)sizeof(io_t) + 32 + 15) / 16) * 16;
     static constexpr bool HAS_Z = GATE && !PHASE1;
     static constexpr bool HAS_C = !PHASE1;
@@ -280,7 +284,7 @@ struct Layout {
     // tensor copies), the rest is packed at 16-byte alignment to keep the CTA's footprint small
     static constexpr int OFF_U = 0;
     static constexpr int OFF_DL = OFF_U + STAGES * ROWS;
-    static constexpr int OFF_Z = OFF_DL + STAGES * ROWS;
+    static constexpr int OFF_Z = OFF_DL + STAGES * ROWS_DL;
     static constexpr int OFF_BR = OFF_Z + (HAS_Z ? STAGES * ROWS : 0);
     static constexpr int OFF_CR = OFF_BR + STAGES * BCRAW;
     static constexpr int OFF_BF = OFF_CR + (HAS_C ? STAGES * BCRAW : 0);  // fp32 B, then fp32 C
@@ -291,7 +295,7 @@ struct Layout {
     static constexpr int OFF_BAR = OFF_OUT + STAGES * OUT_STRIDE;         // full, ready, empty
     static constexpr int OFF_FLAG = OFF_BAR + 3 * STAGES * 8;
     static constexpr int BYTES = OFF_FLAG + 16;
-    static_assert(ROWS % 128 == 0 && BCRAW % 16 == 0 && OFF_BR % 128 == 0 && OFF_BF % 16 == 0 &&
+    static_assert(ROWS % 128 == 0 && ROWS_DL % 128 == 0 && BCRAW % 16 == 0 && OFF_BR % 128 == 0 && OFF_BF % 16 == 0 &&
                       BF_STRIDE % 16 == 0 && OFF_OUT % 8 == 0,
                   "tensor-copy destinations need 128-byte and vector accesses 16-byte alignment");
 };
@@ -305,7 +309,8 @@ struct Layout {
 // Warp 0 refills the stage released two tiles earlier, so kStages-2 tiles are in flight
 // ahead of the one being scanned, and no warp other than warp 0 ever waits for another.
 
-template <typename io_t, int NS, int WARPS, bool GATE, bool PHASE1, bool YPART, bool CONV>
+template <typename io_t, typename dl_t, int NS, int WARPS, bool GATE, bool PHASE1, bool YPART,
+          bool CONV>
 __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     scan_kernel(const __grid_constant__ ScanParams p)
 {
@@ -313,7 +318,9 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     // column-order boxes) keep one more tile in flight; the others keep the ring smaller so
     // that more CTAs fit on an SM (both measured on B200).
     constexpr int kStages = YPART ? 5 : 4;
-    using Lay = Layout<io_t, NS, WARPS, GATE, PHASE1, kStages>;
+    using Lay = Layout<io_t, dl_t, NS, WARPS, GATE, PHASE1, kStages>;
+    // int8 Delta codes: delta_raw = code * delta_scale[d]
+    constexpr bool DQ = std::is_same<dl_t, int8_t>::value;
     // the producer refills the stage released two tiles back and prepares the next tile, so at
     // least four stages are needed for a tile to be in flight while the current one is scanned
     static_assert(kStages >= 4, "the pipeline needs at least four stages");
@@ -411,6 +418,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     const int xmask =
         dir == SS_DIR_REV ? (kTile - 1) : (dir == SS_DIR_COL_REV && umode == 1 ? 7 : 0);
     constexpr uint32_t kBox2 = static_cast<uint32_t>(DC) * kTile * sizeof(io_t);
+    constexpr uint32_t kBoxDL = static_cast<uint32_t>(DC) * kTile * sizeof(dl_t);
     constexpr uint32_t kBox3 = static_cast<uint32_t>(DC) * 8 * sizeof(io_t);
     constexpr uint32_t kUZ = Lay::HAS_Z ? 2u : 1u;
 
@@ -424,7 +432,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
         const void* bsrc = bc_src(gB, t0, rows, bbytes, bskip);
         const void* csrc = Lay::HAS_C ? bc_src(gC, t0, rows, cbytes, cskip) : nullptr;
         if (lane == 0) {
-            uint32_t tx = kBox2 + bbytes + cbytes;  // delta box, B, C
+            uint32_t tx = kBoxDL + bbytes + cbytes;  // delta box, B, C
             if (umode == 0)
                 tx += kUZ * kBox2;
             else if (umode == 1)
@@ -432,7 +440,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
             else
                 tx += kUZ * static_cast<uint32_t>(rows) * row_bytes;
             mbar_expect_tx(&full[st], tx);
-            tma_2d(smem + Lay::OFF_DL + st * Lay::ROWS, &p.tm_dl, static_cast<int32_t>(d0),
+            tma_2d(smem + Lay::OFF_DL + st * Lay::ROWS_DL, &p.tm_dl, static_cast<int32_t>(d0),
                    static_cast<int32_t>(kb * p.L + t0), &full[st]);
             if (umode == 0) {
                 // reverse order: the box ends at the row of step t0
@@ -531,6 +539,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     float a_l[NS];       // A[d, n] (natural units; multiplies Delta*log2(e))
     bool chain = true;   // A[d, n] == (n+1) * A[d, 0] for all n
     float dskip = 0.f, bias2 = 0.f, bias_raw = 0.f;
+    float dscale = 1.f, dscale2 = kLog2e;  // int8 codes: scale[d], and scale[d] * log2(e)
     if (active) {
 #pragma unroll
         for (int n = 0; n < NS; ++n) {
@@ -541,6 +550,10 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
         dskip = p.Dskip ? p.Dskip[d] : 0.f;
         bias_raw = p.bias ? p.bias[d] : 0.f;
         bias2 = bias_raw * kLog2e;
+        if (DQ) {
+            dscale = p.delta_scale[d];
+            dscale2 = dscale * kLog2e;
+        }
     } else {
 #pragma unroll
         for (int n = 0; n < NS; ++n)
@@ -691,7 +704,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
 
         if (active) {
             const io_t* su = reinterpret_cast<const io_t*>(smem + Lay::OFF_U + st * Lay::ROWS);
-            const io_t* sdl = reinterpret_cast<const io_t*>(smem + Lay::OFF_DL + st * Lay::ROWS);
+            const dl_t* sdl = reinterpret_cast<const dl_t*>(smem + Lay::OFF_DL + st * Lay::ROWS_DL);
             const io_t* sz = reinterpret_cast<const io_t*>(smem + Lay::OFF_Z + st * Lay::ROWS);
             const int32_t* orow = reinterpret_cast<const int32_t*>(smem + Lay::OFF_OUT + st * Lay::OUT_STRIDE);
             float* yp_out = p.ypart ? p.ypart + out_base + tid : nullptr;
@@ -706,8 +719,8 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
                 for (int r = 0; r < rows; ++r) {
                     const float uv =
                         conv_step(Io<io_t>::ld(su + (r ^ xmask) * DC + tid), std::true_type{});
-                    const float dr = Io<io_t>::ld(sdl + r * DC + tid);
-                    const float x = dr + bias_raw;
+                    const float dr = Io<dl_t>::ld(sdl + r * DC + tid);
+                    const float x = DQ ? fmaf(dr, dscale, bias_raw) : dr + bias_raw;
                     const float spv = fmaxf(x, 0.f) + log1p_unit(ex2(-fabsf(x) * kLog2e));
                     const float dt = softplus ? spv : x;
                     const float w = dt * uv;
@@ -764,9 +777,9 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
                         // in the segment's last tile)
                         const float uv =
                             conv_step(Io<io_t>::ld(su + (r ^ xmask) * DC + tid), std::false_type{});
-                        const float dr = Io<io_t>::ld(sdl + r * DC + tid);
+                        const float dr = Io<dl_t>::ld(sdl + r * DC + tid);
                         // x = (delta + bias) * log2(e); Delta*log2(e) = softplus in base 2 of x
-                        const float x = fmaf(dr, kLog2e, bias2);
+                        const float x = fmaf(dr, DQ ? dscale2 : kLog2e, bias2);
                         const float e = ex2(-fabsf(x));              // 2^-|x| in (0, 1]
                         const float l_big = lg2(1.f + e);
                         // log2(1+e) for small e: e*log2(e)*(1 - e/2), rel. error < e^2/3
@@ -1004,23 +1017,31 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 
 // A row-major tensor of `rank` dims (innermost first) with element strides `pitch` bytes for
 // dims 1.., read in boxes `box`; out-of-range elements read as zero.
-bool encode(CUtensorMap* map, const void* base, bool bf16, int rank, const cuuint64_t* dims,
-            const cuuint64_t* pitch, const cuuint32_t* box)
+template <typename T> constexpr CUtensorMapDataType map_type()
+{
+    return sizeof(T) == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8  // int8 codes, reinterpreted in the kernel
+           : sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+}
+
+bool encode(CUtensorMap* map, const void* base, CUtensorMapDataType type, int rank,
+            const cuuint64_t* dims, const cuuint64_t* pitch, const cuuint32_t* box)
 {
     PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
     if (!fn)
         return false;
     const cuuint32_t unit[3] = {1, 1, 1};
-    return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+    return fn(map, type,
               static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, pitch, box, unit,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename io_t>
+template <typename io_t, typename dl_t>
 cudaError_t make_maps(ScanParams& p, bool need_z)
 {
-    constexpr bool bf16 = sizeof(io_t) == 2;
+    constexpr CUtensorMapDataType ty = map_type<io_t>();
+    constexpr CUtensorMapDataType ty_dl = map_type<dl_t>();
     const cuuint64_t esz = sizeof(io_t);
     const cuuint64_t D = static_cast<cuuint64_t>(p.D);
     const cuuint32_t box2[2] = {static_cast<cuuint32_t>(32 * kWarps), static_cast<cuuint32_t>(kTile)};
@@ -1029,9 +1050,10 @@ cudaError_t make_maps(ScanParams& p, bool need_z)
     const cuuint64_t dims_kbl[2] = {D, static_cast<cuuint64_t>(p.K * p.batch * p.L)};
     const int64_t u_blocks = p.u_per_dir ? p.K * p.batch : p.batch;  // row blocks of u
     const cuuint64_t dims_u[2] = {D, static_cast<cuuint64_t>(u_blocks * p.L)};
-    if (!encode(&p.tm_u, p.u, bf16, 2, dims_u, pitch2, box2) ||
-        !encode(&p.tm_dl, p.delta, bf16, 2, dims_kbl, pitch2, box2) ||
-        (need_z && !encode(&p.tm_z, p.z, bf16, 2, dims_bl, pitch2, box2)))
+    const cuuint64_t pitch_dl[1] = {D * sizeof(dl_t)};
+    if (!encode(&p.tm_u, p.u, ty, 2, dims_u, pitch2, box2) ||
+        !encode(&p.tm_dl, p.delta, ty_dl, 2, dims_kbl, pitch_dl, box2) ||
+        (need_z && !encode(&p.tm_z, p.z, ty, 2, dims_bl, pitch2, box2)))
         return cudaErrorInvalidValue;
     bool col = false;
     for (int k = 0; k < p.K; ++k)
@@ -1044,20 +1066,20 @@ cudaError_t make_maps(ScanParams& p, bool need_z)
                                      static_cast<cuuint64_t>(p.batch * p.H)};
         const cuuint64_t dims3u[3] = {D, static_cast<cuuint64_t>(p.W),
                                       static_cast<cuuint64_t>(u_blocks * p.H)};
-        if (!encode(&p.tm_u3, p.u, bf16, 3, dims3u, pitch3, box3) ||
-            (need_z && !encode(&p.tm_z3, p.z, bf16, 3, dims3, pitch3, box3)))
+        if (!encode(&p.tm_u3, p.u, ty, 3, dims3u, pitch3, box3) ||
+            (need_z && !encode(&p.tm_z3, p.z, ty, 3, dims3, pitch3, box3)))
             return cudaErrorInvalidValue;
     }
     return cudaSuccess;
 }
 
-template <typename io_t, int NS, bool GATE, bool PHASE1, bool YPART, bool CONV>
+template <typename io_t, typename dl_t, int NS, bool GATE, bool PHASE1, bool YPART, bool CONV>
 cudaError_t launch_t(const ScanParams& p0, cudaStream_t stream)
 {
-    using Lay = Layout<io_t, NS, kWarps, GATE, PHASE1, YPART ? 5 : 4>;
-    auto kern = scan_kernel<io_t, NS, kWarps, GATE, PHASE1, YPART, CONV>;
+    using Lay = Layout<io_t, dl_t, NS, kWarps, GATE, PHASE1, YPART ? 5 : 4>;
+    auto kern = scan_kernel<io_t, dl_t, NS, kWarps, GATE, PHASE1, YPART, CONV>;
     ScanParams p = p0;
-    cudaError_t e = make_maps<io_t>(p, Lay::HAS_Z);
+    cudaError_t e = make_maps<io_t, dl_t>(p, Lay::HAS_Z);
     if (e != cudaSuccess)
         return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::BYTES);
@@ -1075,32 +1097,33 @@ cudaError_t launch_t(const ScanParams& p0, cudaStream_t stream)
                      after_aggregates, p);
 }
 
-template <typename io_t, int NS, bool CONV>
+template <typename io_t, typename dl_t, int NS, bool CONV>
 cudaError_t launch_nc(const ScanParams& p, int phase1, cudaStream_t stream)
 {
     if (phase1)
-        return launch_t<io_t, NS, false, true, false, CONV>(p, stream);
+        return launch_t<io_t, dl_t, NS, false, true, false, CONV>(p, stream);
     if (p.ypart)
-        return launch_t<io_t, NS, false, false, true, CONV>(p, stream);
-    return p.z ? launch_t<io_t, NS, true, false, false, CONV>(p, stream)
-               : launch_t<io_t, NS, false, false, false, CONV>(p, stream);
+        return launch_t<io_t, dl_t, NS, false, false, true, CONV>(p, stream);
+    return p.z ? launch_t<io_t, dl_t, NS, true, false, false, CONV>(p, stream)
+               : launch_t<io_t, dl_t, NS, false, false, false, CONV>(p, stream);
 }
 
-template <typename io_t, int NS>
+template <typename io_t, typename dl_t, int NS>
 cudaError_t launch_ns(const ScanParams& p, int phase1, cudaStream_t stream)
 {
-    return p.conv_w ? launch_nc<io_t, NS, true>(p, phase1, stream)
-                    : launch_nc<io_t, NS, false>(p, phase1, stream);
+    return p.conv_w ? launch_nc<io_t, dl_t, NS, true>(p, phase1, stream)
+                    : launch_nc<io_t, dl_t, NS, false>(p, phase1, stream);
 }
 
-template <typename io_t>
+// All scan launches of io type io_t with delta stored as dl_t (io_t, or int8_t codes).
+template <typename io_t, typename dl_t = io_t>
 cudaError_t launch_io(const ScanParams& p, int phase1, cudaStream_t stream)
 {
     if (p.N <= 4)
-        return launch_ns<io_t, 4>(p, phase1, stream);
+        return launch_ns<io_t, dl_t, 4>(p, phase1, stream);
     if (p.N <= 8)
-        return launch_ns<io_t, 8>(p, phase1, stream);
-    return launch_ns<io_t, 16>(p, phase1, stream);
+        return launch_ns<io_t, dl_t, 8>(p, phase1, stream);
+    return launch_ns<io_t, dl_t, 16>(p, phase1, stream);
 }
 
 }  // namespace

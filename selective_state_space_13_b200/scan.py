@@ -26,6 +26,7 @@ SS_FLAG_GENERIC_A = 1
 SS_FLAG_ZOH_EXACT = 2
 SS_FLAG_TEST_WAIT_TIMEOUT = 8
 SS_FLAG_U_PER_DIRECTION = 16
+SS_FLAG_DELTA_INT8 = 32
 SS_ERR_DEVICE_TIMEOUT = 9
 SS_MAX_DSTATE = 16
 SS_MAX_DIRS = 4
@@ -57,7 +58,7 @@ class SsLaunchOpts(ctypes.Structure):
                 ("scan_begin_event", ctypes.c_void_p), ("scan_end_event", ctypes.c_void_p),
                 ("initial_state", ctypes.c_void_p), ("conv_weight", ctypes.c_void_p),
                 ("conv_bias", ctypes.c_void_p), ("conv_width", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("reserved", ctypes.c_int32), ("delta_scale", ctypes.c_void_p)]
 
 
 class ScanError(RuntimeError):
@@ -159,18 +160,20 @@ def make_dirmap(dirs=(SS_DIR_FWD,), H=0, W=0) -> SsDirectionMap:
 
 
 def make_opts(segments=0, flags=0, events=None, initial_state=0, conv_weight=0, conv_bias=0,
-              conv_width=0) -> SsLaunchOpts:
+              conv_width=0, delta_scale=0) -> SsLaunchOpts:
     """events: optional (begin, end) torch.cuda.Event pair, recorded by the library around its
     main scan launch on the call's stream (each must have been recorded once before, so that
     its CUDA event exists).  initial_state: device address of a [K, batch, D, N] fp32 array
     (0 = zero state).  conv_weight / conv_bias: device addresses of the [K, D, conv_width] and
-    [K, D] fp32 causal-convolution taps and bias (0 = none)."""
+    [K, D] fp32 causal-convolution taps and bias (0 = none).  delta_scale: device address of
+    the [D] fp32 scales of int8 delta codes (used with SS_FLAG_DELTA_INT8)."""
     o = SsLaunchOpts()
     o.segments, o.flags = int(segments), int(flags)
     o.initial_state = int(initial_state) or None
     o.conv_weight = int(conv_weight) or None
     o.conv_bias = int(conv_bias) or None
     o.conv_width = int(conv_width)
+    o.delta_scale = int(delta_scale) or None
     if events is not None:
         o.scan_begin_event = int(events[0].cuda_event) or None
         o.scan_end_event = int(events[1].cuda_event) or None
@@ -277,7 +280,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
                        dirs=(SS_DIR_FWD,), H=0, W=0, out=None, last_state=None,
                        return_last_state=False, workspace=None, stream=None, segments=0,
                        flags=0, events=None, initial_state=None, zoh_exact=False,
-                       conv_weight=None, conv_bias=None):
+                       conv_weight=None, conv_bias=None, delta_scale=None):
     """Selective scan forward on CUDA tensors.
 
     u, z: [batch, L, D] (u may be [K, batch, L, D]: direction k scans its own input u[k],
@@ -288,7 +291,8 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     Bbar = (exp(Delta*A) - 1) / A * B instead of Delta*B.
     conv_weight: [K, D, width] float32 (width <= 4), the causal depthwise convolution each
     direction applies to u along its own scan order, followed by SiLU (None = no convolution);
-    conv_bias: [K, D] float32 or None.
+    conv_bias: [K, D] float32 or None.  delta may be int8 codes (bfloat16 io only) with
+    delta_scale [D] float32: the raw value is code * delta_scale[d].
     Returns out, or (out, last_state [K, batch, D, N] float32) with return_last_state.
     """
     import torch
@@ -309,7 +313,14 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     io = u.dtype
     _io_code(io)
     _check(u, "u", tuple(u.shape[:-3]) + (batch, L, Dm), io, device)
-    _check(delta, "delta", (K, batch, L, Dm), io, device)
+    if delta.dtype == torch.int8:
+        if delta_scale is None:
+            raise ValueError("int8 delta needs delta_scale")
+        flags = int(flags) | SS_FLAG_DELTA_INT8
+        _check(delta, "delta", (K, batch, L, Dm), torch.int8, device)
+    else:
+        _check(delta, "delta", (K, batch, L, Dm), io, device)
+    _check(delta_scale, "delta_scale", (Dm,), torch.float32, device)
     _check(B, "B", (K, batch, L, N), io, device)
     _check(C, "C", (K, batch, L, N), io, device)
     _check(z, "z", (batch, L, Dm), io, device)
@@ -337,7 +348,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     shape = make_shape(batch, L, Dm, N, _io_code(io))
     dmap = make_dirmap(dirs, H, W)
     opts = make_opts(segments, flags, events, _ptr(initial_state), _ptr(conv_weight),
-                     _ptr(conv_bias), width)
+                     _ptr(conv_bias), width, _ptr(delta_scale))
     nws = selective_scan_workspace_size(shape, dmap, opts)
     if workspace is None and nws > 0:
         workspace = _workspace(nws, device)

@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol():
     assert set(names) == set(scan.EXPORTED), names
     for name in names:
         assert hasattr(lib, name), name
-    assert scan.ss_abi_version() == 3
+    assert scan.ss_abi_version() == 4
 
 
 def test_status_strings():
@@ -125,6 +125,23 @@ def test_input_per_direction_flag_accepted():
     sh = _shape()
     o = scan.make_opts(flags=scan.SS_FLAG_U_PER_DIRECTION)
     assert scan.selective_scan_workspace_size(sh, scan.make_dirmap((0, 0)), o) > 0
+
+
+def test_int8_delta_options_validated():
+    I8 = scan.SS_FLAG_DELTA_INT8
+    ok = scan.make_opts(flags=I8, delta_scale=FAKE)
+    assert scan.selective_scan_workspace_size(_shape(), None, ok) == 0
+    cases = [(_shape(io_dtype=scan.SS_F32), ok, 6),          # int8 delta needs bf16 io
+             (_shape(), scan.make_opts(flags=I8), 1),          # scales missing
+             (_shape(dim=40), ok, 4),                           # code rows not 16-byte multiples
+             (_shape(), scan.make_opts(delta_scale=FAKE), 6)]   # scales without the flag
+    for sh, o, want in cases:
+        with pytest.raises(scan.ScanError) as e:
+            scan.selective_scan_workspace_size(sh, None, o)
+        assert e.value.status == want
+    st = scan.selective_scan_fwd_raw(_shape(), FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, 0, 1, None, FAKE,
+                                     0, 0, 0, 0, scan.make_opts(flags=I8, delta_scale=FAKE + 2))
+    assert st == 4
 
 
 def test_conv_options_validated():

@@ -263,6 +263,29 @@ def test_input_per_direction_row_by_row_columns(cuda_device):
     _check(wl.make_inputs(w), cuda_device)
 
 
+# ----------------------------------------------------------------------------- int8 Delta
+
+@pytest.mark.parametrize("segments", [0, 1, 3])
+def test_int8_delta_single_direction(cuda_device, segments):
+    w = wl.variant("m130", name="i8", batch=2, seqlen=300, dim=144, delta_int8=True, seed=150)
+    _check(wl.make_inputs(w), cuda_device, segments=segments)
+
+
+@pytest.mark.parametrize("N", [4, 8, 16])
+def test_int8_delta_state_sizes_with_conv(cuda_device, N):
+    w = wl.variant("m130", name="i8c", batch=2, seqlen=97, dim=64, dstate=N, delta_int8=True,
+                   conv=4, seed=151 + N)
+    _check(wl.make_inputs(w), cuda_device, segments=2)
+
+
+def test_int8_delta_directions_and_exact_zoh(cuda_device):
+    w = wl.variant("ss2d", name="i8_ss2d", batch=2, seqlen=16 * 6, H=16, W=6, dim=48,
+                   delta_int8=True, seed=156)
+    _check(wl.make_inputs(w), cuda_device)
+    w = wl.variant("vim", name="i8_vim", batch=3, dim=64, delta_int8=True, seed=157)
+    _check(wl.make_inputs(w), cuda_device, segments=2, zoh_exact=True)
+
+
 # ----------------------------------------------------------------------------- full size
 
 FULL_SAMPLES = {
@@ -274,13 +297,17 @@ FULL_SAMPLES = {
     "ss2d": (4, 16),
     "m130_conv": (None, 24),
     "cromb": (4, 16),
+    "m130_int8": (None, 24),
 }
 
+FULL_VARIANTS = {"m130_conv": dict(conv=4), "m130_int8": dict(delta_int8=True)}
 
-@pytest.mark.parametrize("name", ["tiny", "m130", "long", "vim", "ss2d", "m130_conv", "cromb"])
+
+@pytest.mark.parametrize("name", ["tiny", "m130", "long", "vim", "ss2d", "m130_conv", "cromb",
+                                  "m130_int8"])
 def test_full_size_workloads_sampled(cuda_device, name):
     import torch
-    w = wl.variant("m130", conv=4) if name == "m130_conv" else wl.WORKLOADS[name]
+    w = wl.variant("m130", **FULL_VARIANTS[name]) if name in FULL_VARIANTS else wl.WORKLOADS[name]
     inp = wl.make_inputs(w)
     t = to_device(inp, cuda_device)
     out, last = run_gpu(inp, dev_inputs=t)            # default launch = the benchmark's
