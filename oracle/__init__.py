@@ -21,6 +21,8 @@ Readings of the pages that the oracle fixes (each is listed with its reason in t
   * The state starts at zero unless an initial state is given.
   * Delta may arrive as int8 codes q with one scale per channel: the raw value is q * scale[d]
     ("S4 -> Mamba" sec. 2.3; the pages give no scale convention).
+  * A, Dskip and delta_bias may be given per direction ([K, D, N], [K, D], [K, D]): direction k
+    then uses its own (VMamba's cross-scan and Vim's two directions are separate S6 modules).
   * With u given per direction ([K, batch, L, D]), direction k scans its own input; Sigma's
     CroMB ("S4 -> Mamba" sec. 4.1) is two such directions in forward order with the C of the
     other modality, summed.
@@ -69,7 +71,7 @@ def _load():
             lib.ss_oracle_scan.restype = ctypes.c_int
             lib.ss_oracle_scan.argtypes = [i64, i64, i64, i64, i32, dp, i64, i64,
                                            dp, dp, dp, dp, dp, dp, dp, dp,
-                                           i32, i32, dp, dp, i32, dp, dp, dp, i64, i32, dp]
+                                           i32, i32, dp, dp, i32, dp, dp, dp, i64, i32, dp, i32]
             lib.ss_oracle_conv_silu.restype = ctypes.c_int
             lib.ss_oracle_conv_silu.argtypes = [i64, i64, i64, i32, dp, i64, i64, dp, dp, dp,
                                                 i64, dp]
@@ -128,7 +130,8 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
     """Run the oracle.
 
     u, z: [batch, L, D] (u may be [K, batch, L, D]: direction k then reads u[k], as in the
-    cross-modal scan); delta: [K, batch, L, D]; B, C: [K, batch, L, N]; A: [D, N];
+    cross-modal scan); delta: [K, batch, L, D]; B, C: [K, batch, L, N]; A: [D, N], or
+    [K, D, N] for parameters per direction (then Dskip and delta_bias are [K, D]);
     Dskip, delta_bias: [D] or None; initial_state: [K, batch, D, N] or None (zero);
     conv_weight: [K, D, width] or None (u is used as it is); conv_bias: [K, D] or None;
     delta_scale: [D] or None -- with it, delta holds int8 codes q and the raw value is
@@ -147,18 +150,22 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
     if u.ndim not in (3, 4) or (u_per_dir and u.shape[0] != K):
         raise ValueError("u must be [batch, L, D] or [K, batch, L, D]")
     batch, L, D = u.shape[-3:]
-    if A.ndim != 2 or A.shape[0] != D:
-        raise ValueError("A must be [D, N]")
-    N = A.shape[1]
+    params_per_dir = A.ndim == 3
+    if A.ndim not in (2, 3) or A.shape[-2] != D or (params_per_dir and A.shape[0] != K):
+        raise ValueError("A must be [D, N] or [K, D, N]")
+    N = A.shape[-1]
     if delta.shape != (K, batch, L, D):
         raise ValueError("delta must be [K, batch, L, D], got %r" % (delta.shape,))
     if B.shape != (K, batch, L, N) or C.shape != (K, batch, L, N):
         raise ValueError("B and C must be [K, batch, L, N]")
     if z is not None and z.shape != (batch, L, D):
         raise ValueError("z must be [batch, L, D]")
-    for v in (Dskip, delta_bias, delta_scale):
-        if v is not None and v.shape != (D,):
-            raise ValueError("Dskip, delta_bias and delta_scale must be [D]")
+    pshape = (K, D) if params_per_dir else (D,)
+    for v in (Dskip, delta_bias):
+        if v is not None and v.shape != pshape:
+            raise ValueError("Dskip and delta_bias must be %r" % (pshape,))
+    if delta_scale is not None and delta_scale.shape != (D,):
+        raise ValueError("delta_scale must be [D]")
     if initial_state is not None and initial_state.shape != (K, batch, D, N):
         raise ValueError("initial_state must be [K, batch, D, N]")
     if conv_weight is not None:
@@ -175,7 +182,7 @@ def selective_scan(u, delta, A, B, C, Dskip=None, z=None, delta_bias=None, softp
                                 int(bool(zoh_exact)), _ptr(out), _ptr(last), int(threads),
                                 _ptr(initial_state), _ptr(conv_weight), _ptr(conv_bias),
                                 0 if conv_weight is None else int(conv_weight.shape[2]),
-                                int(u_per_dir), _ptr(delta_scale))
+                                int(u_per_dir), _ptr(delta_scale), int(params_per_dir))
     if rc != 0:
         raise ValueError("oracle rejected its arguments (code %d)" % rc)
     return out, last

@@ -40,6 +40,8 @@
  *                                                          sigma(z)*(y_fwd+y_bwd), "Vision Mamba"
  *                                                          sec. 2.2; SS2D merge, "S4 -> Mamba" sec. 3)
  *
+ * With params_per_direction, direction k reads its own A[k], Dskip[k] and delta_bias[k] (VMamba's
+ * cross-scan and Vim's two scan directions are separate S6 modules, each with its own parameters).
  * With u_per_direction, direction k reads its own input u[k] wherever u appears above.  This is
  * the cross-modal scan of Sigma's CroMB ("S4 -> Mamba" sec. 4.1): two modalities, each scanned
  * over its own input with the C of the other modality, outputs summed -- the caller stacks the
@@ -57,8 +59,8 @@
  *   u, z                 [batch, L, D]   spatial order (u: [K, batch, L, D] with u_per_direction)
  *   delta                [K, batch, L, D] scan order of direction k
  *   B, C                 [K, batch, L, N] scan order of direction k
- *   A                    [D, N]
- *   Dskip, delta_bias    [D] or NULL (NULL means zero)
+ *   A                    [D, N] ([K, D, N] with params_per_direction)
+ *   Dskip, delta_bias    [D] ([K, D] with params_per_direction) or NULL (NULL means zero)
  *   z                    NULL means no gate
  *   out                  [batch, L, D]
  *   last_state           [K, batch, D, N] or NULL
@@ -168,7 +170,7 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                    double* out, double* last_state, int32_t nthreads,
                    const double* initial_state, const double* conv_weight,
                    const double* conv_bias, int64_t conv_width, int32_t u_per_direction,
-                   const double* delta_scale)
+                   const double* delta_scale, int32_t params_per_direction)
 {
     int bad = 0;
     if (batch < 0 || L < 0 || D < 0 || N < 1 || K < 1 || K > 4)
@@ -210,6 +212,10 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                 memset(yacc, 0, sizeof(double) * (size_t)L);
                 for (int32_t k = 0; k < K; ++k) {
                     const double* uk = u_per_direction ? u + (int64_t)k * batch * L * D : u;
+                    const int64_t pk = params_per_direction ? (int64_t)k : 0;
+                    const double* Ak = A + pk * D * N;
+                    const double* Dk = Dskip ? Dskip + pk * D : NULL;
+                    const double* biask = delta_bias ? delta_bias + pk * D : NULL;
                     for (int64_t n = 0; n < N; ++n)
                         h[n] = initial_state
                                    ? initial_state[(((int64_t)k * batch + b) * D + d) * N + n]
@@ -226,12 +232,12 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                         const int64_t row = ((int64_t)k * batch + b) * L + t;
                         const double draw = delta_scale ? delta[row * D + d] * delta_scale[d]
                                                         : delta[row * D + d];
-                        double dt = draw + (delta_bias ? delta_bias[d] : 0.0);
+                        double dt = draw + (biask ? biask[d] : 0.0);
                         if (softplus)
                             dt = oracle_softplus(dt);
                         double yt = 0.0;
                         for (int64_t n = 0; n < N; ++n) {
-                            const double a = A[d * N + n];
+                            const double a = Ak[d * N + n];
                             const double abar = exp(dt * a);
                             double bcoef;
                             if (zoh_exact)
@@ -241,7 +247,7 @@ int ss_oracle_scan(int64_t batch, int64_t L, int64_t D, int64_t N, int32_t K,
                             h[n] = abar * h[n] + bcoef * B[row * N + n] * ut;
                             yt += C[row * N + n] * h[n];
                         }
-                        yacc[p] += yt + (Dskip ? Dskip[d] : 0.0) * ut;
+                        yacc[p] += yt + (Dk ? Dk[d] : 0.0) * ut;
                     }
                     if (last_state)
                         for (int64_t n = 0; n < N; ++n)

@@ -15,6 +15,9 @@ Recipe (identical for every workload, seed = 20260 + workload index):
   * Dskip = 1 (fp32), except the tiny workload where Dskip ~ N(0, 1);
   * delta_bias: Delta0 ~ exp(U[ln 1e-3, ln 0.1]) per channel, bias = softplus^-1(Delta0) =
     Delta0 + log(-expm1(-Delta0)); the tiny workload uses bias = 0;
+  * with parameters per direction (`params_per_dir`): A[k, d, n] = -(n + 1) * (1 + k/4),
+    Dskip[k] = 1 + k/4 (or N(0, 1) per direction), delta_bias drawn per direction as above, so
+    that every direction's parameters differ;
   * with int8 Delta (`delta_int8`): delta_raw is drawn as above in float32, then quantised
     symmetrically per channel: scale[d] = max |delta_raw[:, :, :, d]| / 127 over directions,
     batch rows and steps, q = round-half-even(delta_raw / scale[d]) (in [-127, 127]); the
@@ -64,6 +67,7 @@ class Workload:
     conv: int = 0                   # taps of the causal convolution before the scan (0: none)
     u_per_dir: bool = False         # one input u[k] per direction ([K, batch, L, D])
     delta_int8: bool = False        # delta_raw as int8 codes with one fp32 scale per channel
+    params_per_dir: bool = False    # A [K, D, N], Dskip and delta_bias [K, D]
     extra: dict = field(default_factory=dict, compare=False)
 
     @property
@@ -90,7 +94,8 @@ class Workload:
         if self.delta_int8:
             nbytes += self.dim * 4                                 # its scales
         nbytes += 2 * self.K * bln * e                             # B, C per direction
-        nbytes += self.dim * self.dstate * 4 + 2 * self.dim * 4    # A, Dskip, delta_bias
+        nbytes += (self.K if self.params_per_dir else 1) * (self.dim * self.dstate + 2 * self.dim) * 4
+        # A, Dskip, delta_bias
         if with_last_state:
             nbytes += self.K * self.batch * self.dim * self.dstate * 4
         if self.conv:
@@ -208,16 +213,20 @@ def make_inputs(w: Workload | str, threads: int | None = None) -> dict:
     B = np.stack([_normal((b, L, N), ss(3, k), w.dtype, threads) for k in range(K)])
     C = np.stack([_normal((b, L, N), ss(4, k), w.dtype, threads) for k in range(K)])
     g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([root, 5])))
+    P = K if w.params_per_dir else 1               # parameter sets
     if w.dskip == "normal":
-        Dskip = g.standard_normal(D).astype(np.float32)
+        Dskip = g.standard_normal((P, D)).astype(np.float32)
     else:
-        Dskip = np.ones(D, dtype=np.float32)
+        Dskip = np.stack([np.full(D, 1.0 + k / 4.0, dtype=np.float32) for k in range(P)])
     if w.bias == "zero":
-        bias = np.zeros(D, dtype=np.float32)
+        bias = np.zeros((P, D), dtype=np.float32)
     else:
-        d0 = np.exp(g.uniform(math.log(1e-3), math.log(0.1), size=D))
+        d0 = np.exp(g.uniform(math.log(1e-3), math.log(0.1), size=(P, D)))
         bias = (d0 + np.log(-np.expm1(-d0))).astype(np.float32)
-    A = np.tile(-(np.arange(N, dtype=np.float32) + 1.0), (D, 1))
+    A = np.stack([np.tile(-(np.arange(N, dtype=np.float32) + 1.0) * np.float32(1.0 + k / 4.0), (D, 1))
+                  for k in range(P)])
+    if not w.params_per_dir:
+        A, Dskip, bias = A[0], Dskip[0], bias[0]
     conv_weight = conv_bias = None
     if w.conv:
         gc = np.random.Generator(np.random.PCG64(np.random.SeedSequence([root, 6])))
@@ -258,10 +267,10 @@ def inputs_f64(inp: dict, channels=None, batches=None) -> dict:
 
     return dict(u=big(inp["u"], w.u_per_dir), z=big(inp["z"], False), delta=big(inp["delta"], True),
                 B=bc(inp["B"]), C=bc(inp["C"]),
-                A=np.asarray(inp["A"][dsel], dtype=np.float64),
-                Dskip=np.asarray(inp["Dskip"][dsel], dtype=np.float64),
+                A=np.asarray(inp["A"][..., dsel, :], dtype=np.float64),
+                Dskip=np.asarray(inp["Dskip"][..., dsel], dtype=np.float64),
                 delta_bias=None if inp["delta_bias"] is None else
-                np.asarray(inp["delta_bias"][dsel], dtype=np.float64),
+                np.asarray(inp["delta_bias"][..., dsel], dtype=np.float64),
                 conv_weight=None if inp.get("conv_weight") is None else
                 np.asarray(inp["conv_weight"][:, dsel], dtype=np.float64),
                 conv_bias=None if inp.get("conv_bias") is None else

@@ -18,11 +18,11 @@ import tests.test_oracle_pins as pins
 SRC = os.path.join(os.path.dirname(oracle.__file__), "ss_oracle.c")
 
 MUTATIONS = [
-    ("dropped D skip", "(Dskip ? Dskip[d] : 0.0) * ut", "0.0 * ut"),
+    ("dropped D skip", "(Dk ? Dk[d] : 0.0) * ut", "0.0 * ut"),
     ("B read where C belongs", "bcoef * B[row * N + n] * ut", "bcoef * C[row * N + n] * ut"),
     ("C read where B belongs", "yt += C[row * N + n] * h[n]", "yt += B[row * N + n] * h[n]"),
     ("wrong sign in exp(Delta A)", "exp(dt * a)", "exp(-dt * a)"),
-    ("dropped delta bias", "+ (delta_bias ? delta_bias[d] : 0.0)", "+ 0.0"),
+    ("dropped delta bias", "+ (biask ? biask[d] : 0.0)", "+ 0.0"),
     ("softplus skipped", "dt = oracle_softplus(dt);", "dt = dt;"),
     ("softplus sign", "log1p(exp(-fabs(x)))", "log1p(exp(fabs(x)))"),
     ("column map transposed", "return (t % H) * W + (t / H);", "return (t / W) * W + (t % W);"),
@@ -47,17 +47,19 @@ MUTATIONS = [
      "u[(b * L + s) * D + d]"),
     ("conv bias dropped", "double c = bias;", "double c = 0.0;"),
     ("no activation after the conv", "return oracle_silu(c);", "return c;"),
-    ("D skip reads the unconvolved input", "(Dskip ? Dskip[d] : 0.0) * ut;",
-     "(Dskip ? Dskip[d] : 0.0) * u[(b * L + p) * D + d];"),
+    ("D skip reads the unconvolved input", "(Dk ? Dk[d] : 0.0) * ut;",
+     "(Dk ? Dk[d] : 0.0) * u[(b * L + p) * D + d];"),
     ("scan takes conv weights of direction 0", "uk, b, d, L, D, dirs[k], H, W, t,\n"
      "                                      conv_weight + ((int64_t)k * D + d) * conv_width,",
      "uk, b, d, L, D, dirs[k], H, W, t,\n"
      "                                      conv_weight + ((int64_t)0 * D + d) * conv_width,"),
     ("int8 scale of the first channel", "delta[row * D + d] * delta_scale[d]",
      "delta[row * D + d] * delta_scale[0]"),
-    ("int8 scale applied after the bias", "double dt = draw + (delta_bias ? delta_bias[d] : 0.0);",
-     "double dt = (delta_scale ? (delta[row * D + d] + (delta_bias ? delta_bias[d] : 0.0)) * "
-     "delta_scale[d] : draw + (delta_bias ? delta_bias[d] : 0.0));"),
+    ("int8 scale applied after the bias", "double dt = draw + (biask ? biask[d] : 0.0);",
+     "double dt = (delta_scale ? (delta[row * D + d] + (biask ? biask[d] : 0.0)) * "
+     "delta_scale[d] : draw + (biask ? biask[d] : 0.0));"),
+    ("parameters of the first direction for all", "const int64_t pk = params_per_direction ? (int64_t)k : 0;",
+     "const int64_t pk = 0;"),
     ("every direction reads the first input", "u_per_direction ? u + (int64_t)k * batch",
      "u_per_direction ? u + (int64_t)0 * batch"),
 ]

@@ -35,6 +35,8 @@ identity, a special case or a brute force that does not run the oracle's recurre
       scans of those inputs, gated; and Sigma's CroMB ("S4 -> Mamba" sec. 4.1) written as the
       pages give it, SSM(x_rgb, C=C_depth) + SSM(x_depth, C=C_rgb) from two separate scans,
       equals the two-direction scan with the C tensors stacked in swapped order.
+  P13 parameters per direction: a K-direction scan whose directions carry their own A, Dskip and
+      delta_bias equals the sum of K single-direction scans, each with its own parameters, gated.
   P12 int8 Delta ("S4 -> Mamba" sec. 2.3): codes q with one scale per channel scan exactly like
       the raw values q * scale[d] given directly (the products are exact in float64).
   plus the silu gate against sigmoid written out, a hand-worked Abar = 1/2 example, empty and
@@ -571,3 +573,28 @@ def test_P12_int8_delta_codes_with_channel_scales(softplus):
     out2, _ = oracle.selective_scan(c["u"], 2 * q, c["A"], c["B"], c["C"], delta_scale=scale / 2,
                                     **args)
     assert np.array_equal(out2, out)
+
+
+# ----------------------------------------------------------------------------- P13 (parameters per direction)
+
+@pytest.mark.parametrize("dirs,H,W", [((FWD, REV), 1, 21), ((FWD, COL, REV, COLREV), 4, 5)])
+def test_P13_parameters_per_direction(dirs, H, W):
+    rng = np.random.default_rng(99 + len(dirs))
+    batch, L, D, N, K = 2, H * W, 3, 4, len(dirs)
+    c = rand_case(rng, batch, L, D, N, K=K)
+    A = -rng.uniform(0.1, 2.0, size=(K, D, N))
+    Dskip = rng.standard_normal((K, D))
+    bias = rng.uniform(-2.0, 0.5, size=(K, D))
+    out, last = oracle.selective_scan(c["u"], c["delta"], A, c["B"], c["C"], Dskip=Dskip,
+                                      z=c["z"], delta_bias=bias, dirs=dirs, H=H, W=W)
+    total = np.zeros_like(c["u"])
+    lasts = []
+    for k, kind in enumerate(dirs):
+        y_k, l_k = oracle.selective_scan(c["u"], c["delta"][k:k + 1], A[k], c["B"][k:k + 1],
+                                         c["C"][k:k + 1], Dskip=Dskip[k], z=None,
+                                         delta_bias=bias[k], dirs=(kind,), H=H, W=W)
+        total += y_k
+        lasts.append(l_k[0])
+    gate = c["z"] / (1.0 + np.exp(-c["z"]))
+    assert rel_err(out, total * gate) < 1e-13
+    assert np.array_equal(last, np.stack(lasts))
