@@ -140,6 +140,10 @@ typedef struct {
                                  io_dtype SS_BF16 and dim a multiple of 16 (the code rows are
                                  dim bytes; SS_ERR_ALIGN otherwise); the base pointer follows
                                  the 16-byte rule                                        */
+#define SS_FLAG_PARAMS_PER_DIRECTION 64 /* A is [K, D, N], Dskip and delta_bias [K, D]:
+                                           direction k uses its own parameters (VMamba's
+                                           cross-scan and Vim's two directions are separate
+                                           S6 modules); delta_scale stays [D]               */
 #define SS_FLAG_TEST_WAIT_TIMEOUT 8 /* test hook for failure detection: every CTA waits (20 ms
                                        at most) on a barrier that nothing completes, gives up,
                                        records SS_ERR_DEVICE_TIMEOUT for
@@ -160,11 +164,12 @@ ss_status selective_scan_workspace_size(const ss_shape* shape, const ss_directio
  *                                  SS_FLAG_U_PER_DIRECTION)
  *   delta       [K, batch, L, D]   io dtype (int8 codes with SS_FLAG_DELTA_INT8), raw Delta of
  *                                  direction k in its scan order
- *   A           [D, N]             fp32, shared by all directions
+ *   A           [D, N]             fp32, shared by all directions ([K, D, N] with
+ *                                  SS_FLAG_PARAMS_PER_DIRECTION)
  *   B, C        [K, batch, L, N]   io dtype, scan order of direction k
- *   Dskip       [D] fp32, or NULL for zero
+ *   Dskip       [D] fp32 ([K, D] with SS_FLAG_PARAMS_PER_DIRECTION), or NULL for zero
  *   z           [batch, L, D]      io dtype, spatial order, or NULL for no gate
- *   delta_bias  [D] fp32, or NULL for zero
+ *   delta_bias  [D] fp32 ([K, D] with SS_FLAG_PARAMS_PER_DIRECTION), or NULL for zero
  *   softplus    nonzero: Delta = softplus(delta + bias); zero: Delta = delta + bias
  *   dmap        direction map (host pointer), or NULL for a single forward scan
  *   out         [batch, L, D]      io dtype, spatial order; every element written once

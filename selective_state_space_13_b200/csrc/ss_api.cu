@@ -123,7 +123,8 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
         if (opts->segments < 0 || opts->segments > kMaxSegments)
             return SS_ERR_UNSUPPORTED;
         if (opts->flags & ~(SS_FLAG_GENERIC_A | SS_FLAG_ZOH_EXACT | SS_FLAG_TEST_WAIT_TIMEOUT |
-                            SS_FLAG_U_PER_DIRECTION | SS_FLAG_DELTA_INT8))
+                            SS_FLAG_U_PER_DIRECTION | SS_FLAG_DELTA_INT8 |
+                            SS_FLAG_PARAMS_PER_DIRECTION))
             return SS_ERR_UNSUPPORTED;
         if (opts->flags & SS_FLAG_DELTA_INT8) {
             if (s->io_dtype != SS_BF16)
@@ -286,6 +287,7 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
     p.zoh = (pl.flags & SS_FLAG_ZOH_EXACT) ? 1 : 0;
     p.test_timeout = (pl.flags & SS_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
     p.u_per_dir = (pl.flags & SS_FLAG_U_PER_DIRECTION) ? 1 : 0;
+    p.params_per_dir = (pl.flags & SS_FLAG_PARAMS_PER_DIRECTION) ? 1 : 0;
     p.status = ss::status_word();
     if (!p.status)
         return SS_ERR_CUDA;

@@ -24,12 +24,12 @@ struct ScanParams {
     CUtensorMap tm_u3, tm_z3;  // u, z as [batch*H, W, D]: boxes of 8 image rows of one column
     const void* u;          // [batch, L, D] io, spatial order ([K, batch, L, D] with u_per_dir)
     const void* delta;      // [K, batch, L, D] io (or int8 codes), scan order
-    const float* A;         // [D, N]
+    const float* A;         // [D, N] ([K, D, N] with params_per_dir)
     const void* B;          // [K, batch, L, N] io, scan order
     const void* C;          // [K, batch, L, N] io, scan order
-    const float* Dskip;     // [D] or null
+    const float* Dskip;     // [D] ([K, D] with params_per_dir) or null
     const void* z;          // [batch, L, D] io or null
-    const float* bias;      // [D] or null
+    const float* bias;      // [D] ([K, D] with params_per_dir) or null
     void* out;              // [batch, L, D] io (single direction) or null
     float* ypart;           // [K, batch, L, D] fp32 per-direction outputs (several directions)
     float* last_state;      // [K, batch, D, N] or null
@@ -51,6 +51,7 @@ struct ScanParams {
     int32_t test_timeout;   // 1: test hook, wait on a barrier nothing completes and report
     int32_t conv_width;     // taps of conv_w (1..SS_MAX_CONV_WIDTH) when conv_w is set
     int32_t u_per_dir;      // 1: direction k reads its own input u[k]
+    int32_t params_per_dir; // 1: direction k reads its own A[k], Dskip[k], bias[k]
     unsigned int* status;   // the device error word (status_word()), or'ed by bounded waits
 };
 

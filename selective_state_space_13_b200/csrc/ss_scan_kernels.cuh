@@ -541,14 +541,17 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     float dskip = 0.f, bias2 = 0.f, bias_raw = 0.f;
     float dscale = 1.f, dscale2 = kLog2e;  // int8 codes: scale[d], and scale[d] * log2(e)
     if (active) {
+        // parameters of this direction (one set shared by all directions unless per direction)
+        const int64_t pk = p.params_per_dir ? static_cast<int64_t>(k) : 0;
+        const float* Ak = p.A + pk * p.D * p.N;
 #pragma unroll
         for (int n = 0; n < NS; ++n) {
-            a_l[n] = (n < p.N) ? p.A[d * p.N + n] : 0.f;
+            a_l[n] = (n < p.N) ? Ak[d * p.N + n] : 0.f;
             if (n < p.N && a_l[n] != static_cast<float>(n + 1) * a_l[0])
                 chain = false;
         }
-        dskip = p.Dskip ? p.Dskip[d] : 0.f;
-        bias_raw = p.bias ? p.bias[d] : 0.f;
+        dskip = p.Dskip ? p.Dskip[pk * p.D + d] : 0.f;
+        bias_raw = p.bias ? p.bias[pk * p.D + d] : 0.f;
         bias2 = bias_raw * kLog2e;
         if (DQ) {
             dscale = p.delta_scale[d];

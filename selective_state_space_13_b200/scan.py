@@ -27,6 +27,7 @@ SS_FLAG_ZOH_EXACT = 2
 SS_FLAG_TEST_WAIT_TIMEOUT = 8
 SS_FLAG_U_PER_DIRECTION = 16
 SS_FLAG_DELTA_INT8 = 32
+SS_FLAG_PARAMS_PER_DIRECTION = 64
 SS_ERR_DEVICE_TIMEOUT = 9
 SS_MAX_DSTATE = 16
 SS_MAX_DIRS = 4
@@ -285,7 +286,8 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
 
     u, z: [batch, L, D] (u may be [K, batch, L, D]: direction k scans its own input u[k],
     e.g. the two modalities of a cross-modal scan); delta: [K, batch, L, D] (or [batch, L, D] when K = 1); B, C:
-    [K, batch, L, N] (or [batch, L, N]); A: [D, N] float32; D (skip) and delta_bias: [D] float32.
+    [K, batch, L, N] (or [batch, L, N]); A: [D, N] float32; D (skip) and delta_bias: [D] float32
+    (or A [K, D, N], D and delta_bias [K, D]: parameters per direction).
     u, delta, B, C, z share one dtype (float32 or bfloat16); out has that dtype.
     initial_state: [K, batch, D, N] float32 state before step 0 (None = zero); zoh_exact: use
     Bbar = (exp(Delta*A) - 1) / A * B instead of Delta*B.
@@ -310,6 +312,10 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     if C.dim() == 3:
         C = C.unsqueeze(0)
     N = A.shape[-1]
+    pshape = (Dm,)
+    if A.dim() == 3:
+        flags = int(flags) | SS_FLAG_PARAMS_PER_DIRECTION
+        pshape = (K, Dm)
     io = u.dtype
     _io_code(io)
     _check(u, "u", tuple(u.shape[:-3]) + (batch, L, Dm), io, device)
@@ -324,9 +330,9 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     _check(B, "B", (K, batch, L, N), io, device)
     _check(C, "C", (K, batch, L, N), io, device)
     _check(z, "z", (batch, L, Dm), io, device)
-    _check(A, "A", (Dm, N), torch.float32, device)
-    _check(D, "D", (Dm,), torch.float32, device)
-    _check(delta_bias, "delta_bias", (Dm,), torch.float32, device)
+    _check(A, "A", pshape[:-1] + (Dm, N), torch.float32, device)
+    _check(D, "D", pshape, torch.float32, device)
+    _check(delta_bias, "delta_bias", pshape, torch.float32, device)
     if out is None:
         out = torch.empty((batch, L, Dm), dtype=io, device=device)
     _check(out, "out", (batch, L, Dm), io, device)

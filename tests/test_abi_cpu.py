@@ -123,7 +123,7 @@ def test_null_alignment_and_workspace_errors():
 
 def test_input_per_direction_flag_accepted():
     sh = _shape()
-    o = scan.make_opts(flags=scan.SS_FLAG_U_PER_DIRECTION)
+    o = scan.make_opts(flags=scan.SS_FLAG_U_PER_DIRECTION | scan.SS_FLAG_PARAMS_PER_DIRECTION)
     assert scan.selective_scan_workspace_size(sh, scan.make_dirmap((0, 0)), o) > 0
 
 

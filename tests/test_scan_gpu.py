@@ -286,6 +286,25 @@ def test_int8_delta_directions_and_exact_zoh(cuda_device):
     _check(wl.make_inputs(w), cuda_device, segments=2, zoh_exact=True)
 
 
+# ----------------------------------------------------------------------------- parameters per direction
+
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F32])
+def test_parameters_per_direction_vim(cuda_device, dtype):
+    w = wl.variant("vim", name="ppd_vim", batch=3, dim=64, dtype=dtype, params_per_dir=True,
+                   seed=160)
+    _check(wl.make_inputs(w), cuda_device, segments=2)
+
+
+def test_parameters_per_direction_cross_scan_generic_A_conv(cuda_device):
+    w = wl.variant("ss2d", name="ppd_ss2d", batch=2, seqlen=16 * 5, H=16, W=5, dim=32,
+                   params_per_dir=True, conv=4, dskip="normal", seed=161)
+    inp = wl.make_inputs(w)
+    _check(inp, cuda_device)
+    rng = np.random.default_rng(12)
+    inp["A"] = (-rng.uniform(0.05, 3.0, size=inp["A"].shape)).astype(np.float32)
+    _check(inp, cuda_device, segments=3)
+
+
 # ----------------------------------------------------------------------------- full size
 
 FULL_SAMPLES = {
