@@ -11,13 +11,16 @@ namespace {
 
 constexpr int64_t kMaxSeqlen = (int64_t{1} << 31) - 1;
 // Automatic segment choice (measured on B200): when the (direction, batch row, channel tile)
-// units give fewer than about 1.5 CTAs per SM, split each sequence until they reach about 4 per
-// SM, and split long sequences into segments of about kLongSegSteps steps; never below
-// kMinSegSteps steps.  (With more units, the segment-aggregate launch costs more than the
-// parallelism it adds.)
+// units give fewer than about 1.5 CTAs per SM, split each sequence into S segments so that the
+// scan launch's units * S CTAs fill one wave of the kWaveCtas resident slots (6 CTAs on each
+// of the 148 SMs) as closely as possible without starting a second, mostly idle wave; when the
+// segments would still exceed kLongSegSteps steps, S is multiplied up to whole waves again.
+// Segments never go below kMinSegSteps steps.  (With more units the segment-aggregate launch
+// costs more than the parallelism it adds.)  Measured: m130 -> 4, long -> 22, cromb -> 18,
+// 10-15% faster than a fixed target for the last two.
 constexpr int64_t kSplitBelowCtas = 222;
-constexpr int64_t kTargetCtas = 4 * 148;
-constexpr int64_t kLongSegSteps = 4096;
+constexpr int64_t kWaveCtas = 6 * 148;
+constexpr int64_t kLongSegSteps = 8192;
 constexpr int64_t kMinSegSteps = 16 * ss::kTile;
 constexpr int kMaxSegments = 1024;
 
@@ -151,10 +154,10 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
                              pl->batch * pl->K;
         seg = 1;
         if (ctas > 0 && ctas < kSplitBelowCtas) {
-            int64_t want = (kTargetCtas + ctas - 1) / ctas;
-            const int64_t by_len = L / kLongSegSteps;
-            if (want < by_len)
-                want = by_len;
+            int64_t want = kWaveCtas / ctas;  // >= 4: ctas < kSplitBelowCtas
+            const int64_t waves = (L + want * kLongSegSteps - 1) / (want * kLongSegSteps);
+            if (waves > 1)
+                want *= waves;
             const int64_t cap = L / kMinSegSteps;
             if (want > cap)
                 want = cap;
