@@ -366,3 +366,150 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     if st != SS_OK:
         raise ScanError(st, "selective_scan_fwd")
     return (out, last_state) if return_last_state else out
+
+
+# ----------------------------------------------------------------------------- host buffers
+
+_host_streams = {}
+_host_staging = {}
+
+
+def _streams(device):
+    import torch
+    key = device.index
+    if key not in _host_streams:
+        _host_streams[key] = tuple(torch.cuda.Stream(device=device) for _ in range(3))
+    return _host_streams[key]
+
+
+def _slot(name, slot, shape, dtype, device):
+    import torch
+    key = (name, slot, tuple(shape), dtype, device.index)
+    buf = _host_staging.get(key)
+    if buf is None:
+        buf = torch.empty(tuple(shape), dtype=dtype, device=device)
+        _host_staging[key] = buf
+    return buf
+
+
+def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                            dirs=(SS_DIR_FWD,), H=0, W=0, out=None, last_state=None,
+                            return_last_state=False, flags=0, initial_state=None,
+                            zoh_exact=False, conv_weight=None, conv_bias=None, delta_scale=None,
+                            chunks=8, device=None):
+    """Selective scan of inputs held in host memory, with the results written back to host memory.
+
+    u, delta, B, C, z (and out, last_state) are CPU tensors -- pinned, so that the copies are
+    asynchronous -- with the shapes of selective_scan_fwd; A, D, delta_bias, conv_weight,
+    conv_bias, delta_scale and initial_state are parameters already on the device.  The work is
+    cut into `chunks` pieces and pipelined over three streams, so that the host->device copies of
+    one piece, the scan of the previous one and the device->host copy of the one before that run
+    at the same time (the two copy directions use both halves of the duplex host link).  Pieces
+    are groups of batch rows; a single batch row of one forward direction without convolution is
+    cut along the sequence instead, each piece continuing from the previous piece's final state.
+    The scans run in the CUDA library (selective_scan_fwd); the call returns once everything is
+    enqueued, ordered after the caller's current stream, which it rejoins at the end.
+    Returns out, or (out, last_state) with return_last_state.
+    """
+    import torch
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    K = len(dirs)
+    if delta.dim() == 3:
+        delta = delta.unsqueeze(0)
+    if B.dim() == 3:
+        B = B.unsqueeze(0)
+    if C.dim() == 3:
+        C = C.unsqueeze(0)
+    u_per_dir = u.dim() == 4
+    batch, L, Dm = u.shape[-3:]
+    N = A.shape[-1]
+    io = u.dtype
+    if out is None:
+        out = torch.empty((batch, L, Dm), dtype=io, pin_memory=True)
+    want_last = return_last_state or last_state is not None
+    if want_last and last_state is None:
+        last_state = torch.empty((K, batch, Dm, N), dtype=torch.float32, pin_memory=True)
+    seq_split = (batch == 1 and K == 1 and int(dirs[0]) == SS_DIR_FWD and conv_weight is None
+                 and not u_per_dir)
+    total = L if seq_split else batch
+    nch = max(1, min(int(chunks), total))
+    step = -(-total // nch)
+    if seq_split:
+        step = -(-step // 16) * 16  # whole 16-step tiles
+    pieces = [(i, min(total, i + step)) for i in range(0, total, step)] if total else []
+
+    cur = torch.cuda.current_stream(device)
+    s_in, s_comp, s_out = _streams(device)
+    start = torch.cuda.Event()
+    start.record(cur)
+    for s in (s_in, s_comp, s_out):
+        s.wait_event(start)
+    comp_done, out_done = [], []
+    prev_last = initial_state
+    for i, (a, b) in enumerate(pieces):
+        slot = i % 2
+        n = b - a
+        # the piece's views of the host tensors, and device slots of the same shapes
+        if seq_split:
+            views = dict(u=u[:, a:b], delta=delta[:, :, a:b], B=B[:, :, a:b], C=C[:, :, a:b],
+                         z=None if z is None else z[:, a:b])
+            oview = out[:, a:b]
+        else:
+            views = dict(u=u[..., a:b, :, :], delta=delta[:, a:b], B=B[:, a:b], C=C[:, a:b],
+                         z=None if z is None else z[a:b])
+            oview = out[a:b]
+        dev = {k: None if v is None else _slot(k, slot, v.shape, v.dtype, device)
+               for k, v in views.items()}
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(comp_done[i - 2])  # the scan of piece i-2 has read this slot
+            for k, v in views.items():
+                if v is None:
+                    continue
+                if v.dim() == 4 and not v.is_contiguous():  # [K, rows, ...]: one copy per k
+                    for kk in range(v.shape[0]):
+                        dev[k][kk].copy_(v[kk], non_blocking=True)
+                else:
+                    dev[k].copy_(v, non_blocking=True)
+            in_done = torch.cuda.Event()
+            in_done.record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(in_done)
+            if i >= 2:
+                s_comp.wait_event(out_done[i - 2])  # the output slot has been copied out
+            o_dev = _slot("out", slot, oview.shape, io, device)
+            l_dev = _slot("last", slot, (K, 1 if seq_split else n, Dm, N), torch.float32, device) \
+                if (want_last or seq_split) else None
+            if seq_split:
+                h0 = prev_last
+            else:
+                h0 = None if initial_state is None else initial_state[:, a:b].contiguous()
+            selective_scan_fwd(dev["u"], dev["delta"], A, dev["B"], dev["C"], D=D, z=dev["z"],
+                               delta_bias=delta_bias, softplus=softplus, dirs=dirs, H=H, W=W,
+                               out=o_dev, last_state=l_dev, flags=flags, initial_state=h0,
+                               zoh_exact=zoh_exact, conv_weight=conv_weight, conv_bias=conv_bias,
+                               delta_scale=delta_scale, stream=s_comp)
+            prev_last = l_dev
+            done = torch.cuda.Event()
+            done.record(s_comp)
+            comp_done.append(done)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done)
+            oview.copy_(o_dev, non_blocking=True)
+            if want_last and not seq_split:
+                for kk in range(K):
+                    last_state[kk, a:b].copy_(l_dev[kk], non_blocking=True)
+            if want_last and seq_split and i == len(pieces) - 1:
+                last_state.copy_(l_dev, non_blocking=True)
+            od = torch.cuda.Event()
+            od.record(s_out)
+            out_done.append(od)
+    for s in (s_in, s_comp, s_out):
+        ev = torch.cuda.Event()
+        ev.record(s)
+        cur.wait_event(ev)
+    if want_last and not pieces:
+        last_state.copy_(initial_state if initial_state is not None else
+                         torch.zeros_like(last_state))
+    return (out, last_state) if return_last_state else out

@@ -305,6 +305,71 @@ def test_parameters_per_direction_cross_scan_generic_A_conv(cuda_device):
     _check(inp, cuda_device, segments=3)
 
 
+# ----------------------------------------------------------------------------- host buffers
+
+def _host_case(inp, device, chunks=4, initial_state=None):
+    """selective_scan_fwd_host on pinned host copies of the inputs, checked against the oracle."""
+    import torch
+    from selective_state_space_13_b200 import scan
+    w = inp["workload"]
+    t = to_device(inp, device)
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in t.items()}
+    h0 = None if initial_state is None else \
+        torch.from_numpy(np.ascontiguousarray(initial_state, dtype=np.float32)).to(device)
+    out, last = scan.selective_scan_fwd_host(
+        host["u"], host["delta"], t["A"], host["B"], host["C"], D=t["D"], z=host["z"],
+        delta_bias=t["delta_bias"], softplus=w.softplus, dirs=w.dirs, H=w.H, W=w.W,
+        return_last_state=True, initial_state=h0, conv_weight=t["conv_weight"],
+        conv_bias=t["conv_bias"], delta_scale=t["delta_scale"], chunks=chunks)
+    torch.cuda.synchronize()
+    assert out.device.type == "cpu" and last.device.type == "cpu"
+    ref_out, ref_last = run_oracle(inp, initial_state=initial_state)
+    tol = tol_for(w)
+    e_out, e_last = rel_err(out_to_f64(out), ref_out), rel_err(out_to_f64(last), ref_last)
+    assert e_out <= tol and e_last <= tol, (w.name, e_out, e_last)
+
+
+@pytest.mark.parametrize("chunks", [1, 3, 8])
+def test_host_buffers_batch_pieces(cuda_device, chunks):
+    w = wl.variant("m130", name="host_b", batch=5, seqlen=200, dim=72, seed=170)
+    _host_case(wl.make_inputs(w), cuda_device, chunks=chunks)
+
+
+def test_host_buffers_sequence_pieces(cuda_device):
+    # one batch row of one forward direction: pieces along the sequence, chained by the state
+    w = wl.variant("long", name="host_l", seqlen=1000, dim=64, seed=171)
+    h0 = np.random.default_rng(13).standard_normal((1, 1, 64, 16)).astype(np.float32)
+    _host_case(wl.make_inputs(w), cuda_device, chunks=5, initial_state=h0)
+
+
+def test_host_buffers_sequence_pieces_fp32_exact(cuda_device):
+    # fp32 keeps the state itself, so pieces of whole tiles continued through the stored final
+    # state must reproduce one unsplit scan bit for bit
+    import torch
+    from selective_state_space_13_b200 import scan
+    w = wl.variant("long", name="host_l32", seqlen=1000, dim=64, dtype=wl.F32, seed=171)
+    inp = wl.make_inputs(w)
+    t = to_device(inp, cuda_device)
+    h0 = torch.from_numpy(np.random.default_rng(13).standard_normal((1, 1, 64, 16))
+                          .astype(np.float32)).to(cuda_device)
+    ref, ref_last = scan.selective_scan_fwd(t["u"], t["delta"], t["A"], t["B"], t["C"], D=t["D"],
+                                            z=t["z"], delta_bias=t["delta_bias"],
+                                            return_last_state=True, segments=1, initial_state=h0)
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in t.items()}
+    out, last = scan.selective_scan_fwd_host(host["u"], host["delta"], t["A"], host["B"], host["C"],
+                                             D=t["D"], z=host["z"], delta_bias=t["delta_bias"],
+                                             return_last_state=True, initial_state=h0, chunks=5)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref.cpu()) and torch.equal(last, ref_last.cpu())
+
+
+def test_host_buffers_directions_inputs_and_conv(cuda_device):
+    w = wl.variant("cromb", name="host_c", batch=3, seqlen=150, dim=32, conv=4, seed=172)
+    _host_case(wl.make_inputs(w), cuda_device, chunks=2)
+    w = wl.variant("vim", name="host_v", batch=4, dim=64, delta_int8=True, seed=173)
+    _host_case(wl.make_inputs(w), cuda_device, chunks=3)
+
+
 # ----------------------------------------------------------------------------- full size
 
 FULL_SAMPLES = {
