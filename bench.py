@@ -41,7 +41,6 @@ FLUSH_BYTES = 256 << 20
 # FP32 work of one state update in the form the kernels compute (the exp(Delta*A) of a state
 # taken as one multiply of the power chain, the state multiply-add, the readout multiply-add)
 FLOP_PER_UPDATE = 5
-E2E_PIECES = 8  # pieces of the end-to-end host-buffer pipeline
 # workloads whose description states that last_state is returned
 RETURNS_LAST_STATE = {"tiny", "long"}
 
@@ -366,7 +365,7 @@ def run_ours(args):
                 delta_bias=t["delta_bias"], softplus=w.softplus, dirs=w.dirs, H=w.H, W=w.W,
                 out=out_host, last_state=last_host if last is not None else None,
                 flags=args.flags, conv_weight=t["conv_weight"], conv_bias=t["conv_bias"],
-                delta_scale=t["delta_scale"], chunks=E2E_PIECES)
+                delta_scale=t["delta_scale"], chunks=args.e2e_pieces)
 
         e2e_step()
         torch.cuda.synchronize(device)
@@ -381,7 +380,7 @@ def run_ours(args):
                "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                "ms_per_step": e2e_ms, "steps": n_e2e,
                "path": "selective_scan_fwd_host: pinned host inputs -> device, scan, device -> "
-                       "pinned host, in %d pieces overlapped on 3 streams" % E2E_PIECES}
+                       "pinned host, in %d pieces overlapped on 3 streams" % args.e2e_pieces}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0 at N = 1 only)
     cpu = None
@@ -458,6 +457,8 @@ def parse(argv=None):
                     help="taps of a causal depthwise conv1d + SiLU fused before the scan (0 = none)")
     ap.add_argument("--delta-int8", action="store_true",
                     help="Delta as int8 codes with one scale per channel")
+    ap.add_argument("--e2e-pieces", type=int, default=8,
+                    help="pieces of the end-to-end host-buffer pipeline")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-updates", type=float, default=4e9,
