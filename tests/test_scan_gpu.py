@@ -12,6 +12,8 @@ inputs, <= 2e-2 for bf16 inputs with fp32 state.
 import numpy as np
 import pytest
 
+import oracle
+
 from selective_state_space_13_b200 import workloads as wl
 from tests.scan_util import (TOL_BF16, TOL_F32, out_to_f64, rel_err, run_gpu, run_oracle,
                              to_device, tol_for)
@@ -411,3 +413,43 @@ def test_full_size_workloads_sampled(cuda_device, name):
     del t, out, last, got, got_last
     torch.cuda.empty_cache()
     assert e_out <= tol and e_last <= tol, (name, e_out, e_last)
+
+
+# ----------------------------------------------------------------------------- largest offsets
+
+def test_largest_row_offsets(cuda_device):
+    # L * D just under the 2^31 the ABI allows (1 x 1048576 x 2040 bf16, 4.3 GB per tensor): the
+    # kernels' 32-bit row offsets and tensor-map coordinates at their limit.  The inputs are
+    # drawn on the device from a seeded generator (the host generator would take minutes); the
+    # oracle receives the exact stored values of a few channels.
+    import torch
+    from selective_state_space_13_b200 import scan
+    L, D, N = 1 << 20, 2040, 16
+    assert L * D < 2 ** 31 and L * D > 2 ** 31 - 2 ** 24
+    g = torch.Generator(device=cuda_device).manual_seed(2031)
+
+    def normal(*shape):
+        return torch.randn(shape, generator=g, device=cuda_device).to(torch.bfloat16)
+
+    u, z, delta = normal(1, L, D), normal(1, L, D), normal(1, 1, L, D)
+    B, C = normal(1, 1, L, N), normal(1, 1, L, N)
+    A = -torch.arange(1, N + 1, device=cuda_device, dtype=torch.float32).repeat(D, 1)
+    Dskip = torch.ones(D, device=cuda_device)
+    d0 = torch.exp(torch.empty(D, device=cuda_device).uniform_(np.log(1e-3), np.log(0.1),
+                                                                generator=g))
+    bias = d0 + torch.log(-torch.expm1(-d0))
+    out, last = scan.selective_scan_fwd(u, delta, A, B, C, D=Dskip, z=z, delta_bias=bias,
+                                        return_last_state=True)
+    torch.cuda.synchronize()
+    assert scan.selective_scan_device_status() == scan.SS_OK
+    ch = torch.tensor([0, 1, 1023, 2038, 2039], device=cuda_device)  # both ends of the rows
+    f64 = lambda x: x.double().cpu().numpy()  # noqa: E731
+    ref_out, ref_last = oracle.selective_scan(
+        f64(u.index_select(2, ch)), f64(delta.index_select(3, ch)), f64(A.index_select(0, ch)),
+        f64(B), f64(C), Dskip=f64(Dskip.index_select(0, ch)), z=f64(z.index_select(2, ch)),
+        delta_bias=f64(bias.index_select(0, ch)))
+    e_out = rel_err(f64(out.index_select(2, ch)), ref_out)
+    e_last = rel_err(f64(last.index_select(2, ch)), ref_last)
+    del u, z, delta, out
+    torch.cuda.empty_cache()
+    assert e_out <= TOL_BF16 and e_last <= TOL_BF16, (e_out, e_last)
