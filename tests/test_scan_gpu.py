@@ -453,3 +453,65 @@ def test_largest_row_offsets(cuda_device):
     del u, z, delta, out
     torch.cuda.empty_cache()
     assert e_out <= TOL_BF16 and e_last <= TOL_BF16, (e_out, e_last)
+
+
+# ----------------------------------------------------------------------------- guard bands
+
+GUARD_CASES = {
+    "one_dir_segments": (wl.variant("m130", name="g1", batch=3, seqlen=333, dim=136, seed=180),
+                         dict(segments=5)),
+    "two_dirs": (wl.variant("vim", name="g2", batch=3, seqlen=77, dim=72, seed=181), {}),
+    "cross_scan_rows": (wl.variant("ss2d", name="g3", batch=2, seqlen=10 * 7, H=10, W=7, dim=40,
+                                   seed=182), dict(segments=2)),
+    "conv_int8_per_dir_u": (wl.variant("cromb", name="g4", batch=2, seqlen=150, dim=48, conv=3,
+                                       delta_int8=True, seed=183), dict(segments=3)),
+    "fp32_zoh": (wl.variant("m130", name="g5", batch=2, seqlen=45, dim=20, dtype=wl.F32,
+                            seed=184), dict(zoh_exact=True)),
+}
+
+
+@pytest.mark.parametrize("case", sorted(GUARD_CASES))
+def test_outputs_written_once_inside_their_bounds(cuda_device, case):
+    # out, last_state and the workspace sit inside larger buffers whose margins hold a canary;
+    # out and last_state start as NaN.  After the call every output element must have been
+    # written (no NaN left) and no margin byte changed.
+    import torch
+    from selective_state_space_13_b200 import scan
+    w, kw = GUARD_CASES[case]
+    inp = wl.make_inputs(w)
+    t = to_device(inp, cuda_device)
+    io = t["u"].dtype
+    pad = 64  # elements; keeps every base 16-byte aligned
+
+    def guarded(shape, dtype, canary):
+        n = int(np.prod(shape))
+        buf = torch.full((pad + n + pad,), canary, dtype=dtype, device=cuda_device)
+        view = buf[pad:pad + n].view(shape)
+        view.fill_(float("nan"))
+        return buf, view
+
+    ob, out = guarded((w.batch, w.seqlen, w.dim), io, -8192.0)
+    lb, last = guarded((w.K, w.batch, w.dim, w.dstate), torch.float32, -8192.0)
+    shape = scan.make_shape(w.batch, w.seqlen, w.dim, w.dstate,
+                            scan.SS_BF16 if w.dtype == wl.BF16 else scan.SS_F32)
+    # (the options that change the workspace are the direction map and the segments)
+    nws = scan.selective_scan_workspace_size(shape, scan.make_dirmap(w.dirs, w.H, w.W),
+                                             scan.make_opts(kw.get("segments", 0)))
+    wpad = 256
+    wb = torch.full((wpad + nws + wpad,), 0xA5, dtype=torch.uint8, device=cuda_device)
+    ws = wb[wpad:wpad + nws] if nws else None
+    scan.selective_scan_fwd(t["u"], t["delta"], t["A"], t["B"], t["C"], D=t["D"], z=t["z"],
+                            delta_bias=t["delta_bias"], softplus=w.softplus, dirs=w.dirs, H=w.H,
+                            W=w.W, out=out, last_state=last, workspace=ws,
+                            conv_weight=t["conv_weight"], conv_bias=t["conv_bias"],
+                            delta_scale=t["delta_scale"], **kw)
+    torch.cuda.synchronize()
+    assert scan.selective_scan_device_status() == scan.SS_OK
+    assert not torch.isnan(out.float()).any() and not torch.isnan(last).any()
+    for buf in (ob, lb):
+        assert bool((buf[:pad] == -8192.0).all()) and bool((buf[-pad:] == -8192.0).all())
+    assert bool((wb[:wpad] == 0xA5).all()) and bool((wb[-wpad:] == 0xA5).all())
+    # and the results are the scan's
+    ref_out, ref_last = run_oracle(inp, zoh_exact=kw.get("zoh_exact", False))
+    tol = tol_for(w)
+    assert rel_err(out_to_f64(out), ref_out) <= tol and rel_err(out_to_f64(last), ref_last) <= tol
