@@ -95,18 +95,18 @@ def kernel_source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per launch of the scan kernel from the committed ncu summary, or None when
-    the kernel sources changed since the counters were taken."""
+def recorded_counters(workload: str) -> dict:
+    """The committed ncu record of the scan pipeline for this workload (DRAM bytes and warp
+    instructions per step), or {} when the kernel sources changed since it was taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as fh:
             rec = json.load(fh).get(workload)
     except (OSError, ValueError):
-        return None
+        return {}
     if not rec or rec.get("source_digest") != kernel_source_digest():
-        return None
-    return rec.get("dram_bytes_per_launch")
+        return {}
+    return rec
 
 
 class ClockSampler:
@@ -397,8 +397,20 @@ def run_ours(args):
                          "(%.3g state updates)" % (len(channels), w.dim, w.seqlen, w.K,
                                                    w.updates() * frac)}
 
-    traffic = None if args.seqlen else recorded_traffic(
+    counters = {} if args.seqlen else recorded_counters(
         w.name + ("_conv%d" % w.conv if w.conv else "") + ("_int8" if w.delta_int8 else ""))
+    traffic = counters.get("dram_bytes_per_launch")
+    # instruction issue: the kernels are bound by it (see the counters summaries); achieved =
+    # the recorded warp instructions of one pass over the live pass time, against one warp
+    # instruction per clock on each of the 148 x 4 schedulers
+    issue = None
+    if counters.get("warp_instructions_per_launch"):
+        issue_peak = 148 * 4 * sm_mhz * 1e6 / 1e12
+        issue_ach = counters["warp_instructions_per_launch"] / (kern_ms * 1e-3) / 1e12
+        issue = {"achieved": issue_ach, "peak": issue_peak, "unit": "T warp-instructions/s",
+                 "frac": issue_ach / issue_peak,
+                 "warp_instructions_per_launch": counters["warp_instructions_per_launch"],
+                 "source": "ncu smsp__inst_executed.sum, profiles/traffic.json"}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
@@ -428,7 +440,8 @@ def run_ours(args):
                      "kernel_ms": kern_ms,
                      "hbm": {"achieved": achieved, "peak": peak, "unit": "GB/s",
                              "frac": achieved / peak, "peak_source": peak_src,
-                             "algorithmic_bytes_per_launch": nbytes}},
+                             "algorithmic_bytes_per_launch": nbytes},
+                     "issue": issue},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": sampler.report(),
         "e2e": e2e,
