@@ -383,13 +383,19 @@ def _streams(device):
 
 
 def _slot(name, slot, shape, dtype, device):
+    """A device staging buffer of `shape`: a view of one allocation per (name, slot, dtype,
+    device), grown to the largest piece requested so far (so memory stays bounded by two pieces
+    per tensor, whatever shapes the calls use)."""
     import torch
-    key = (name, slot, tuple(shape), dtype, device.index)
+    key = (name, slot, dtype, device.index)
+    n = 1
+    for e in shape:
+        n *= int(e)
     buf = _host_staging.get(key)
-    if buf is None:
-        buf = torch.empty(tuple(shape), dtype=dtype, device=device)
+    if buf is None or buf.numel() < n:
+        buf = torch.empty(max(n, 1), dtype=dtype, device=device)
         _host_staging[key] = buf
-    return buf
+    return buf[:n].view(tuple(shape))
 
 
 def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
