@@ -515,3 +515,36 @@ def test_outputs_written_once_inside_their_bounds(cuda_device, case):
     ref_out, ref_last = run_oracle(inp, zoh_exact=kw.get("zoh_exact", False))
     tol = tol_for(w)
     assert rel_err(out_to_f64(out), ref_out) <= tol and rel_err(out_to_f64(last), ref_last) <= tol
+
+
+# ----------------------------------------------------------------------------- decoding step by step
+
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F32])
+def test_step_by_step_decoding_matches_one_scan(cuda_device, dtype):
+    # the recurrent form at inference ("Understanding Mamba from zero" sec. 2.3): one step per
+    # call, the state carried through initial_state / last_state, equals one scan of all steps
+    import torch
+    from selective_state_space_13_b200 import scan
+    w = wl.variant("m130", name="decode", batch=4, seqlen=5, dim=256, dtype=dtype, seed=190)
+    inp = wl.make_inputs(w)
+    t = to_device(inp, cuda_device)
+    h = torch.zeros((1, w.batch, w.dim, w.dstate), dtype=torch.float32, device=cuda_device)
+    outs = []
+    for s in range(w.seqlen):
+        o, h = scan.selective_scan_fwd(
+            t["u"][:, s:s + 1].contiguous(), t["delta"][:, :, s:s + 1].contiguous(), t["A"],
+            t["B"][:, :, s:s + 1].contiguous(), t["C"][:, :, s:s + 1].contiguous(), D=t["D"],
+            z=t["z"][:, s:s + 1].contiguous(), delta_bias=t["delta_bias"], initial_state=h,
+            return_last_state=True)
+        outs.append(o)
+    out = torch.cat(outs, dim=1)
+    torch.cuda.synchronize()
+    ref_out, ref_last = run_oracle(inp)
+    tol = tol_for(w)
+    assert rel_err(out_to_f64(out), ref_out) <= tol and rel_err(out_to_f64(h), ref_last) <= tol
+    if dtype == wl.F32:
+        # fp32 keeps h itself: the steps reproduce one unsplit scan bit for bit
+        full, last = scan.selective_scan_fwd(t["u"], t["delta"], t["A"], t["B"], t["C"], D=t["D"],
+                                             z=t["z"], delta_bias=t["delta_bias"], segments=1,
+                                             return_last_state=True)
+        assert torch.equal(out, full) and torch.equal(h, last)
