@@ -10,6 +10,12 @@ once, out written once, parameters and last_state) / device time, summed over ra
 torchrun every rank runs the whole workload on its own GPU (independent problems, weak
 scaling, no collective on the data path); the step time is the max over ranks.
 
+The JSON line also carries: roofline (FP32 FLOP/s of the scan pipeline against the FP32 peak,
+with the HBM fraction and the instruction-issue fraction beside it; DRAM traffic and warp
+instructions per step come from the committed ncu record while the kernel sources match it),
+e2e (the public host-buffer call selective_scan_fwd_host, copies included), clocks (NVML during
+the timed region), gpu_launches and cpu_baseline (the oracle on the host cores).
+
 --impl reference runs the fp64 CPU oracle on a bounded sample of the same workload on the host
 cores (there is no other implementation of this path to compare with).
 """

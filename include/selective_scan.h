@@ -43,6 +43,9 @@
  *     dim * sizeof(io element) must be a multiple of 16 (SS_ERR_ALIGN otherwise).
  *   - N (dstate) is at most SS_MAX_DSTATE; at most SS_MAX_DIRS directions.
  *   - There is no CPU fallback: without a CUDA device every launch returns SS_ERR_CUDA.
+ *   - The first selective_scan_fwd call on each device looks up the address of the library's
+ *     device error word (cudaGetSymbolAddress, once); make that first call before capturing a
+ *     stream into a CUDA graph.
  */
 #ifndef SELECTIVE_SCAN_H
 #define SELECTIVE_SCAN_H

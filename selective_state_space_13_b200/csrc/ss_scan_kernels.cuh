@@ -4,13 +4,15 @@
 // N-state vector in registers for the whole segment ("Understanding Mamba from zero" sec. 5:
 // per channel and per state the recurrence is the scalar affine map h_t = a_t h_{t-1} + b_t).
 // A CTA of 32*WARPS threads owns a tile of adjacent channels.  Its inputs stream through a
-// ring of 4-5 shared-memory stages of kTile steps each; warp 0 fills the ring with bulk
-// asynchronous copies (TMA, cp.async.bulk) that complete on an mbarrier, one copy per row of
-// u / z (rows picked through the direction's index map) and delta (scan order), plus one copy
-// each for the B and C tiles, which every channel of the CTA shares.  B and C are converted to
-// fp32 once per CTA per stage.  Everything of a step -- softplus, exp, the recurrence, the C
-// readout, the D skip and the silu gate -- happens in registers; each input element is read
-// from HBM once and each output element written once.
+// ring of 4-5 shared-memory stages of kTile steps each, filled by asynchronous bulk copies
+// that complete on mbarriers: one tensor-map box (cp.async.bulk.tensor) per tile for u, z and
+// delta (rows picked through the direction's index map: a 2D box for the row orders, 3D boxes
+// of 8 image rows for the column orders, one bulk copy per row otherwise), plus one bulk copy
+// each for the B and C tiles, which every channel of the CTA shares.  The producer duty
+// (refilling the ring, converting B and C to fp32 once per tile) rotates over the warps.
+// Everything of a step -- the optional causal convolution of u, softplus, exp, the recurrence,
+// the C readout, the D skip and the silu gate -- happens in registers; each input element is
+// read from HBM once and each output element written once.
 //
 // Two algebraic rewrites keep the per-update work at three FP32 operations:
 //  * exp-power chain: when A[d,n] = (n+1) * A[d,0] for every n (checked in the kernel, per
@@ -22,7 +24,8 @@
 //    2^-64*|B| in absolute value.
 //  All exponentials run in base 2: x is carried as (delta+bias)*log2(e), so softplus in base 2
 //  gives Delta*log2(e) directly, exp(Delta*A) = ex2(Delta*log2(e) * A), and the missing ln 2
-//  of w = Delta*u is folded into the fp32 copy of B.
+//  of w = Delta*u is folded into the fp32 copy of B.  fp32 inputs (and the exact-ZOH Bbar) take
+//  a precise path instead: h = expm1(Delta*A)*h + (h + Bbar*u*B).
 //
 // Long sequences are split into S segments (the chunked scan of "S4 -> Mamba" sec. 2.2): a
 // first launch scans segments 0..S-2 from a zero state and stores each end state and the
@@ -30,12 +33,17 @@
 // folding the carries of segments 0..s-1 with the affine combine (P2, h2) o (P1, h1) =
 // (P2*P1, P2*h1 + h2), P = exp(A * sum Delta).
 //
+// Options: an initial state, the exact ZOH Bbar, a causal depthwise convolution + SiLU of u per
+// direction, int8 delta codes with per-channel scales, an input and/or a parameter set per
+// direction (see include/selective_scan.h).
+//
 // Every wait on an mbarrier is bounded in time.  A wait that gives up sets the library's device
 // error word (read by selective_scan_device_status), waits a bounded time for the copies this
 // CTA still has in flight, and the whole CTA returns.
 //
-// This header holds the kernels and their launch templates; ss_scan_f32.cu and ss_scan_bf16.cu
-// instantiate them per io type (compiled in parallel), ss_scan.cu holds the host entry points.
+// This header holds the kernels and their launch templates; ss_scan_f32.cu, ss_scan_bf16.cu and
+// ss_scan_bf16_i8.cu instantiate them per io type and delta storage (compiled in parallel), and
+// ss_scan.cu holds the host entry points.
 #pragma once
 
 #include <cuda.h>
@@ -302,12 +310,15 @@ struct Layout {
 
 // ---------------------------------------------------------------------------- the scan kernel
 //
-// Pipeline of one CTA (WARPS warps, every warp scans; warp 0 also produces):
+// Pipeline of one CTA (WARPS warps, every warp scans; in iteration it, warp it % WARPS also
+// produces):
 //   full[s]  completes when the bulk copies of the tile in stage s have landed (tx count);
-//   ready[s] completes when warp 0 has converted that tile's B and C to fp32;
+//   ready[s] completes when the producing warp has converted that tile's B and C to fp32;
 //   empty[s] completes when all WARPS warps are done with the tile in stage s.
-// Warp 0 refills the stage released two tiles earlier, so kStages-2 tiles are in flight
-// ahead of the one being scanned, and no warp other than warp 0 ever waits for another.
+// The producer of iteration it converts tile it+1 (whose copies were issued earlier) and
+// refills the stage released by tile it-2 with tile it+kStages-2, so kStages-2 tiles are in
+// flight ahead of the one being scanned; only the producer ever waits on another warp (for the
+// stage it refills), so the pipeline cannot deadlock.
 
 template <typename io_t, typename dl_t, int NS, int WARPS, bool GATE, bool PHASE1, bool YPART,
           bool CONV>
@@ -422,7 +433,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     constexpr uint32_t kBox3 = static_cast<uint32_t>(DC) * 8 * sizeof(io_t);
     constexpr uint32_t kUZ = Lay::HAS_Z ? 2u : 1u;
 
-    // Fill the stage of time tile `it` (warp 0).
+    // Fill the stage of time tile `it` (called by the producing warp).
     auto issue = [&](int64_t it) {
         const int st = static_cast<int>(it % kStages);
         const int64_t t0 = t_begin + it * kTile;
@@ -487,7 +498,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
             mbar_arrive(&full[st]);
     };
 
-    // Convert tile `it`'s B (and C) to fp32 (warp 0).  On the fast path B carries the ln 2 of
+    // Convert tile `it`'s B (and C) to fp32 (producing warp).  On the fast path B carries the ln 2 of
     // w = Delta*u / ln 2.
     auto convert = [&](int64_t it) {
         const int st = static_cast<int>(it % kStages);
