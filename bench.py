@@ -92,13 +92,40 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier pool measurement)", {}
 
 
+def code_without_comments(text: str) -> str:
+    """C/C++/CUDA source with comments, trailing spaces and blank lines removed (string and
+    character literals kept), so that edits to comments alone keep the digest."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    lines = [ln.rstrip() for ln in "".join(out).splitlines()]
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_digest() -> str:
+    """Digest of the CUDA library's code (sources and headers, comments ignored): the ncu
+    record in profiles/traffic.json applies only while it matches."""
     from selective_state_space_13_b200 import build as b
     h = hashlib.sha256()
     for f in b.SOURCES + b.HEADERS:
-        with open(f, "rb") as fh:
+        with open(f, encoding="utf-8") as fh:
             h.update(os.path.basename(f).encode())
-            h.update(fh.read())
+            h.update(code_without_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
