@@ -548,3 +548,57 @@ def test_step_by_step_decoding_matches_one_scan(cuda_device, dtype):
                                              z=t["z"], delta_bias=t["delta_bias"], segments=1,
                                              return_last_state=True)
         assert torch.equal(out, full) and torch.equal(h, last)
+
+
+# ----------------------------------------------------------------------------- random combinations
+
+def _random_case(i):
+    """A seeded random combination of shape and options, within what the ABI accepts."""
+    rng = np.random.default_rng(5000 + i)
+    dtype = wl.BF16 if rng.random() < 0.7 else wl.F32
+    int8 = dtype == wl.BF16 and rng.random() < 0.3
+    step = 16 if int8 else (8 if dtype == wl.BF16 else 4)
+    D = int(step * rng.integers(1, 200 // step + 1))
+    kind = rng.integers(0, 4)
+    if kind == 0:
+        dirs, H, W = (wl.DIR_FORWARD,), 0, 0
+        L = int(rng.integers(1, 400))
+    elif kind == 1:
+        dirs, H, W = (wl.DIR_FORWARD, wl.DIR_REVERSE), 0, 0
+        L = int(rng.integers(1, 300))
+    else:
+        H, W = int(rng.integers(1, 20)), int(rng.integers(1, 20))
+        L = H * W
+        pool = [wl.DIR_FORWARD, wl.DIR_REVERSE, wl.DIR_COLUMN, wl.DIR_COLUMN_REVERSE]
+        dirs = tuple(int(d) for d in rng.choice(pool, size=int(rng.integers(1, 5)),
+                                                replace=bool(rng.random() < 0.3)))
+    w = wl.Workload("rand%d" % i, int(rng.integers(1, 4)), L, D, int(rng.integers(1, 17)), dtype,
+                    dirs=dirs, H=H, W=W, gate=bool(rng.random() < 0.6),
+                    softplus=bool(rng.random() < 0.85),
+                    bias="zero" if rng.random() < 0.2 else "loguniform",
+                    dskip="normal" if rng.random() < 0.5 else "one", seed=6000 + i,
+                    conv=int(rng.integers(1, 5)) if rng.random() < 0.3 else 0,
+                    u_per_dir=bool(len(dirs) > 1 and rng.random() < 0.3), delta_int8=int8,
+                    params_per_dir=bool(len(dirs) > 1 and rng.random() < 0.3))
+    kw = dict(segments=int(rng.choice([0, 1, 2, 3, 7])))
+    if rng.random() < 0.25:
+        kw["initial_state"] = rng.standard_normal((w.K, w.batch, w.dim, w.dstate)).astype(np.float32)
+    if rng.random() < 0.15:
+        kw["zoh_exact"] = True
+    if rng.random() < 0.1:
+        kw["use_D"] = False
+    return w, kw
+
+
+@pytest.mark.parametrize("i", range(120))
+def test_random_option_combinations(cuda_device, i):
+    w, kw = _random_case(i)
+    inp = wl.make_inputs(w)
+    if not w.softplus:
+        # Delta = delta_raw + bias must stay positive without softplus: the bias of each channel
+        # (and direction) is raised above the largest |delta_raw| it meets
+        raw = wl.inputs_f64(inp)["delta"]                       # [K, b, L, D] raw values
+        need = np.abs(raw).max(axis=(1, 2)) + 0.01                 # [K, D]
+        bias = need.max(axis=0) if inp["delta_bias"].ndim == 1 else need
+        inp["delta_bias"] = bias.astype(np.float32)
+    _check(inp, cuda_device, **kw)
