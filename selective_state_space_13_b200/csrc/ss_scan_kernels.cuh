@@ -847,8 +847,9 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
                                 cp[j] = make_float2(rr * ex2(sp2 * a_l[2 * j]),
                                                     rr * ex2(sp2 * a_l[2 * j + 1]));
                         }
-                        // C . k in two packed accumulators (fewer adds at the end than four)
-                        float2 yacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                        // C . k in two packed accumulators (fewer adds at the end than four),
+                        // started by the products of the first four states (no zeroing)
+                        float2 yacc[2];
 #pragma unroll
                         for (int n4 = 0; n4 < NS / 4; ++n4) {
                             const float4 bq = B4[r * (NS / 4) + n4];
@@ -858,17 +859,21 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
                                                           make_float2(bq.z, bq.w));
                             if (!PHASE1) {
                                 const float4 cq = C4[r * (NS / 4) + n4];
-                                yacc[0] = __ffma2_rn(make_float2(cq.x, cq.y),
-                                                                kst2[2 * n4], yacc[0]);
-                                yacc[1] =
-                                    __ffma2_rn(make_float2(cq.z, cq.w), kst2[2 * n4 + 1],
-                                               yacc[1]);
+                                if (n4 == 0) {
+                                    yacc[0] = __fmul2_rn(make_float2(cq.x, cq.y), kst2[0]);
+                                    yacc[1] = __fmul2_rn(make_float2(cq.z, cq.w), kst2[1]);
+                                } else {
+                                    yacc[0] = __ffma2_rn(make_float2(cq.x, cq.y),
+                                                         kst2[2 * n4], yacc[0]);
+                                    yacc[1] = __ffma2_rn(make_float2(cq.z, cq.w),
+                                                         kst2[2 * n4 + 1], yacc[1]);
+                                }
                             }
                         }
                         if (!PHASE1) {
                             const float2 ys = __fadd2_rn(yacc[0], yacc[1]);
                             float y = fmaf(s_w[g], ys.x + ys.y, s_du[g]);
-                            if (r < rows) {
+                            if (FULL || r < rows) {
                                 if (YPART) {
                                     yp_out[orow[r]] = y;
                                 } else {
