@@ -398,6 +398,19 @@ def _slot(name, slot, shape, dtype, device):
     return buf[:n].view(tuple(shape))
 
 
+def _check_host(t, name, shape, dtype):
+    if t is None:
+        return
+    if t.is_cuda:
+        raise ValueError("%s must be a host (CPU) tensor" % name)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
 def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                             dirs=(SS_DIR_FWD,), H=0, W=0, out=None, last_state=None,
                             return_last_state=False, flags=0, initial_state=None,
@@ -411,9 +424,10 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
     cut into `chunks` pieces and pipelined over three streams, so that the host->device copies of
     one piece, the scan of the previous one and the device->host copy of the one before that run
     at the same time (the two copy directions use both halves of the duplex host link).  Pieces
-    are groups of batch rows; a single batch row of one forward direction without convolution is
-    cut along the sequence instead, each piece continuing from the previous piece's final state.
-    The scans run in the CUDA library (selective_scan_fwd); the call returns once everything is
+    are groups of batch rows; a scan of one forward direction without convolution asked for more
+    pieces than it has batch rows cuts each row along the sequence instead, each piece continuing
+    from the previous piece's final state.  The arguments are checked once; each piece's scan is
+    one selective_scan_fwd call of the CUDA library.  The call returns once everything is
     enqueued, ordered after the caller's current stream, which it rejoins at the end.
     Returns out, or (out, last_state) with return_last_state.
     """
@@ -428,22 +442,82 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
     if C.dim() == 3:
         C = C.unsqueeze(0)
     u_per_dir = u.dim() == 4
+    if u_per_dir and u.shape[0] != K:
+        raise ValueError("u must be [batch, L, D] or [K, batch, L, D]")
     batch, L, Dm = u.shape[-3:]
     N = A.shape[-1]
     io = u.dtype
+    io_code = _io_code(io)
+    if u_per_dir:
+        flags = int(flags) | SS_FLAG_U_PER_DIRECTION
+    pshape = (Dm,)
+    if A.dim() == 3:
+        flags = int(flags) | SS_FLAG_PARAMS_PER_DIRECTION
+        pshape = (K, Dm)
+    if zoh_exact:
+        flags = int(flags) | SS_FLAG_ZOH_EXACT
+    # ---- every argument is checked once here; the pieces below only slice
+    _check_host(u, "u", tuple(u.shape[:-3]) + (batch, L, Dm), io)
+    if delta.dtype == torch.int8:
+        if delta_scale is None:
+            raise ValueError("int8 delta needs delta_scale")
+        flags = int(flags) | SS_FLAG_DELTA_INT8
+        _check_host(delta, "delta", (K, batch, L, Dm), torch.int8)
+    else:
+        _check_host(delta, "delta", (K, batch, L, Dm), io)
+    _check_host(B, "B", (K, batch, L, N), io)
+    _check_host(C, "C", (K, batch, L, N), io)
+    _check_host(z, "z", (batch, L, Dm), io)
+    _check(A, "A", pshape[:-1] + (Dm, N), torch.float32, device)
+    _check(D, "D", pshape, torch.float32, device)
+    _check(delta_bias, "delta_bias", pshape, torch.float32, device)
+    _check(delta_scale, "delta_scale", (Dm,), torch.float32, device)
+    _check(initial_state, "initial_state", (K, batch, Dm, N), torch.float32, device)
+    width = 0
+    if conv_weight is not None:
+        if conv_weight.dim() != 3:
+            raise ValueError("conv_weight must be [K, D, width]")
+        width = int(conv_weight.shape[2])
+        _check(conv_weight, "conv_weight", (K, Dm, width), torch.float32, device)
+    elif conv_bias is not None:
+        raise ValueError("conv_bias needs conv_weight")
+    _check(conv_bias, "conv_bias", (K, Dm), torch.float32, device)
     if out is None:
         out = torch.empty((batch, L, Dm), dtype=io, pin_memory=True)
+    _check_host(out, "out", (batch, L, Dm), io)
     want_last = return_last_state or last_state is not None
     if want_last and last_state is None:
         last_state = torch.empty((K, batch, Dm, N), dtype=torch.float32, pin_memory=True)
-    seq_split = (batch == 1 and K == 1 and int(dirs[0]) == SS_DIR_FWD and conv_weight is None
-                 and not u_per_dir)
-    total = L if seq_split else batch
-    nch = max(1, min(int(chunks), total))
-    step = -(-total // nch)
-    if seq_split:
+    _check_host(last_state, "last_state", (K, batch, Dm, N), torch.float32)
+
+    # ---- pieces (r0, r1, a, b): batch rows r0..r1-1, steps a..b-1
+    nch = max(1, int(chunks))
+    carry = (K == 1 and int(dirs[0]) == SS_DIR_FWD and conv_weight is None and not u_per_dir
+             and L > 0 and (batch == 1 or nch > batch))
+    if carry:
+        parts = -(-nch // batch)
+        step = -(-L // parts)
         step = -(-step // 16) * 16  # whole 16-step tiles
-    pieces = [(i, min(total, i + step)) for i in range(0, total, step)] if total else []
+        pieces = [(r, r + 1, a, min(L, a + step)) for r in range(batch) for a in range(0, L, step)]
+    else:
+        nb = max(1, min(nch, batch))
+        rstep = -(-batch // nb) if batch else 1
+        pieces = [(r, min(batch, r + rstep), 0, L) for r in range(0, batch, rstep)]
+    if L == 0 or Dm == 0:
+        pieces = []
+
+    # ---- the C structures: one direction map, a shape per distinct piece size, and the
+    # workspace of the largest piece
+    dmap = make_dirmap(dirs, H, W)
+    shapes = {}
+    for r0, r1, a, b in pieces:
+        key = (r1 - r0, b - a)
+        if key not in shapes:
+            shapes[key] = make_shape(key[0], key[1], Dm, N, io_code)
+    p_conv_w, p_conv_b, p_scale = _ptr(conv_weight), _ptr(conv_bias), _ptr(delta_scale)
+    probe = make_opts(0, flags, None, 0, p_conv_w, p_conv_b, width, p_scale)
+    nws = max([selective_scan_workspace_size(sh, dmap, probe) for sh in shapes.values()] + [0])
+    p_A, p_D, p_bias = _ptr(A), _ptr(D), _ptr(delta_bias)
 
     cur = torch.cuda.current_stream(device)
     s_in, s_comp, s_out = _streams(device)
@@ -451,20 +525,20 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
     start.record(cur)
     for s in (s_in, s_comp, s_out):
         s.wait_event(start)
+    with torch.cuda.stream(s_comp):
+        ws = _workspace(nws, device) if nws > 0 else None
+    p_ws, n_ws = _ptr(ws), (0 if ws is None else ws.numel())
+    h_comp = s_comp.cuda_stream
     comp_done, out_done = [], []
-    prev_last = initial_state
-    for i, (a, b) in enumerate(pieces):
+    prev_last = None
+    for i, (r0, r1, a, b) in enumerate(pieces):
         slot = i % 2
-        n = b - a
+        rows, steps = r1 - r0, b - a
         # the piece's views of the host tensors, and device slots of the same shapes
-        if seq_split:
-            views = dict(u=u[:, a:b], delta=delta[:, :, a:b], B=B[:, :, a:b], C=C[:, :, a:b],
-                         z=None if z is None else z[:, a:b])
-            oview = out[:, a:b]
-        else:
-            views = dict(u=u[..., a:b, :, :], delta=delta[:, a:b], B=B[:, a:b], C=C[:, a:b],
-                         z=None if z is None else z[a:b])
-            oview = out[a:b]
+        views = dict(u=u[..., r0:r1, a:b, :], delta=delta[:, r0:r1, a:b],
+                     B=B[:, r0:r1, a:b], C=C[:, r0:r1, a:b],
+                     z=None if z is None else z[r0:r1, a:b])
+        oview = out[r0:r1, a:b]
         dev = {k: None if v is None else _slot(k, slot, v.shape, v.dtype, device)
                for k, v in views.items()}
         with torch.cuda.stream(s_in):
@@ -485,17 +559,23 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
             if i >= 2:
                 s_comp.wait_event(out_done[i - 2])  # the output slot has been copied out
             o_dev = _slot("out", slot, oview.shape, io, device)
-            l_dev = _slot("last", slot, (K, 1 if seq_split else n, Dm, N), torch.float32, device) \
-                if (want_last or seq_split) else None
-            if seq_split:
+            l_dev = _slot("last", slot, (K, rows, Dm, N), torch.float32, device) \
+                if (want_last or carry) else None
+            if carry and a > 0:
                 h0 = prev_last
+            elif initial_state is not None:
+                h0 = initial_state[:, r0:r1]
+                if not h0.is_contiguous():
+                    h0 = h0.contiguous()
             else:
-                h0 = None if initial_state is None else initial_state[:, a:b].contiguous()
-            selective_scan_fwd(dev["u"], dev["delta"], A, dev["B"], dev["C"], D=D, z=dev["z"],
-                               delta_bias=delta_bias, softplus=softplus, dirs=dirs, H=H, W=W,
-                               out=o_dev, last_state=l_dev, flags=flags, initial_state=h0,
-                               zoh_exact=zoh_exact, conv_weight=conv_weight, conv_bias=conv_bias,
-                               delta_scale=delta_scale, stream=s_comp)
+                h0 = None
+            opts = make_opts(0, flags, None, _ptr(h0), p_conv_w, p_conv_b, width, p_scale)
+            st = selective_scan_fwd_raw(shapes[(rows, steps)], _ptr(dev["u"]), _ptr(dev["delta"]),
+                                        p_A, _ptr(dev["B"]), _ptr(dev["C"]), p_D, _ptr(dev["z"]),
+                                        p_bias, softplus, dmap, _ptr(o_dev), _ptr(l_dev), p_ws,
+                                        n_ws, h_comp, opts)
+            if st != SS_OK:
+                raise ScanError(st, "selective_scan_fwd")
             prev_last = l_dev
             done = torch.cuda.Event()
             done.record(s_comp)
@@ -503,11 +583,9 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
         with torch.cuda.stream(s_out):
             s_out.wait_event(done)
             oview.copy_(o_dev, non_blocking=True)
-            if want_last and not seq_split:
+            if want_last and b == L:
                 for kk in range(K):
-                    last_state[kk, a:b].copy_(l_dev[kk], non_blocking=True)
-            if want_last and seq_split and i == len(pieces) - 1:
-                last_state.copy_(l_dev, non_blocking=True)
+                    last_state[kk, r0:r1].copy_(l_dev[kk], non_blocking=True)
             od = torch.cuda.Event()
             od.record(s_out)
             out_done.append(od)

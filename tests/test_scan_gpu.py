@@ -365,6 +365,37 @@ def test_host_buffers_sequence_pieces_fp32_exact(cuda_device):
     assert torch.equal(out, ref.cpu()) and torch.equal(last, ref_last.cpu())
 
 
+def test_host_buffers_rows_and_sequence_pieces(cuda_device):
+    # more pieces than batch rows, one forward direction: every row is cut along the sequence,
+    # each piece continuing from the previous piece of its row
+    w = wl.variant("m130", name="host_rs", batch=3, seqlen=700, dim=48, seed=174)
+    h0 = np.random.default_rng(14).standard_normal((1, 3, 48, 16)).astype(np.float32)
+    _host_case(wl.make_inputs(w), cuda_device, chunks=7, initial_state=h0)
+    _host_case(wl.make_inputs(w), cuda_device, chunks=4)
+
+
+def test_host_buffers_rows_and_sequence_pieces_fp32_exact(cuda_device):
+    # pieces of whole tiles per row, chained through the stored final state, reproduce one
+    # unsplit fp32 scan bit for bit
+    import torch
+    from selective_state_space_13_b200 import scan
+    w = wl.variant("m130", name="host_rs32", batch=2, seqlen=1000, dim=64, dtype=wl.F32,
+                   seed=175)
+    inp = wl.make_inputs(w)
+    t = to_device(inp, cuda_device)
+    h0 = torch.from_numpy(np.random.default_rng(15).standard_normal((1, 2, 64, 16))
+                          .astype(np.float32)).to(cuda_device)
+    ref, ref_last = scan.selective_scan_fwd(t["u"], t["delta"], t["A"], t["B"], t["C"], D=t["D"],
+                                            z=t["z"], delta_bias=t["delta_bias"],
+                                            return_last_state=True, segments=1, initial_state=h0)
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in t.items()}
+    out, last = scan.selective_scan_fwd_host(host["u"], host["delta"], t["A"], host["B"], host["C"],
+                                             D=t["D"], z=host["z"], delta_bias=t["delta_bias"],
+                                             return_last_state=True, initial_state=h0, chunks=6)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref.cpu()) and torch.equal(last, ref_last.cpu())
+
+
 def test_host_buffers_directions_inputs_and_conv(cuda_device):
     w = wl.variant("cromb", name="host_c", batch=3, seqlen=150, dim=32, conv=4, seed=172)
     _host_case(wl.make_inputs(w), cuda_device, chunks=2)
