@@ -372,6 +372,8 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
 
 _host_streams = {}
 _host_staging = {}
+# per (device, slot): the event after the last scan that read the slot's staging inputs
+_host_slot_read = {}
 
 
 def _streams(device):
@@ -395,6 +397,7 @@ def _slot(name, slot, shape, dtype, device):
     if buf is None or buf.numel() < n:
         buf = torch.empty(max(n, 1), dtype=dtype, device=device)
         _host_staging[key] = buf
+        _host_slot_read.pop((device.index, slot), None)  # new memory: order after the caller
     return buf[:n].view(tuple(shape))
 
 
@@ -428,7 +431,10 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
     pieces than it has batch rows cuts each row along the sequence instead, each piece continuing
     from the previous piece's final state.  The arguments are checked once; each piece's scan is
     one selective_scan_fwd call of the CUDA library.  The call returns once everything is
-    enqueued, ordered after the caller's current stream, which it rejoins at the end.
+    enqueued, ordered after the caller's current stream, which it rejoins at the end; only its
+    host->device copies start earlier, as soon as the previous call's scans have released the
+    device staging buffers, so that consecutive calls overlap.  The staging buffers and streams
+    are shared by all calls on a device: make those calls from one thread.
     Returns out, or (out, last_state) with return_last_state.
     """
     import torch
@@ -519,11 +525,32 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
     nws = max([selective_scan_workspace_size(sh, dmap, probe) for sh in shapes.values()] + [0])
     p_A, p_D, p_bias = _ptr(A), _ptr(D), _ptr(delta_bias)
 
+    # the staging slots of every piece (allocated or grown here, before any copy is enqueued)
+    views_of, devs_of = [], []
+    for i, (r0, r1, a, b) in enumerate(pieces):
+        views = dict(u=u[..., r0:r1, a:b, :], delta=delta[:, r0:r1, a:b],
+                     B=B[:, r0:r1, a:b], C=C[:, r0:r1, a:b],
+                     z=None if z is None else z[r0:r1, a:b])
+        views_of.append(views)
+        devs_of.append({k: None if v is None else _slot(k, i % 2, v.shape, v.dtype, device)
+                        for k, v in views.items()})
+
     cur = torch.cuda.current_stream(device)
     s_in, s_comp, s_out = _streams(device)
     start = torch.cuda.Event()
     start.record(cur)
-    for s in (s_in, s_comp, s_out):
+    # The scans and the copies back follow the caller's stream.  The copies in only write the
+    # staging slots: they wait for the last scan of the previous call that read each slot, so
+    # that they overlap the end of that call (a slot whose memory is new waits for the caller).
+    for slot in range(min(2, len(pieces))):
+        ev = _host_slot_read.get((device.index, slot))
+        if ev is None:
+            s_in.wait_event(start)
+            break
+    else:
+        for slot in range(min(2, len(pieces))):
+            s_in.wait_event(_host_slot_read[(device.index, slot)])
+    for s in (s_comp, s_out):
         s.wait_event(start)
     with torch.cuda.stream(s_comp):
         ws = _workspace(nws, device) if nws > 0 else None
@@ -535,12 +562,8 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
         slot = i % 2
         rows, steps = r1 - r0, b - a
         # the piece's views of the host tensors, and device slots of the same shapes
-        views = dict(u=u[..., r0:r1, a:b, :], delta=delta[:, r0:r1, a:b],
-                     B=B[:, r0:r1, a:b], C=C[:, r0:r1, a:b],
-                     z=None if z is None else z[r0:r1, a:b])
+        views, dev = views_of[i], devs_of[i]
         oview = out[r0:r1, a:b]
-        dev = {k: None if v is None else _slot(k, slot, v.shape, v.dtype, device)
-               for k, v in views.items()}
         with torch.cuda.stream(s_in):
             if i >= 2:
                 s_in.wait_event(comp_done[i - 2])  # the scan of piece i-2 has read this slot
@@ -589,6 +612,8 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
             od = torch.cuda.Event()
             od.record(s_out)
             out_done.append(od)
+    for i in range(max(0, len(pieces) - 2), len(pieces)):
+        _host_slot_read[(device.index, i % 2)] = comp_done[i]
     for s in (s_in, s_comp, s_out):
         ev = torch.cuda.Event()
         ev.record(s)

@@ -396,6 +396,36 @@ def test_host_buffers_rows_and_sequence_pieces_fp32_exact(cuda_device):
     assert torch.equal(out, ref.cpu()) and torch.equal(last, ref_last.cpu())
 
 
+def test_host_buffers_back_to_back_calls(cuda_device):
+    # consecutive calls without a synchronisation in between, each with its own inputs and
+    # outputs: the copies of a call may start while the previous call's last scans still run,
+    # and every call must still see only its own inputs
+    import torch
+    from selective_state_space_13_b200 import scan
+    w = wl.variant("m130", name="host_bb", batch=4, seqlen=300, dim=64, seed=176)
+    cases = []
+    for j in range(4):
+        inp = wl.make_inputs(wl.variant("m130", name="host_bb%d" % j, batch=4, seqlen=300, dim=64,
+                                        seed=176 + j))
+        t = to_device(inp, cuda_device)
+        ref = scan.selective_scan_fwd(t["u"], t["delta"], t["A"], t["B"], t["C"], D=t["D"],
+                                      z=t["z"], delta_bias=t["delta_bias"])
+        host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in t.items()}
+        cases.append((t, host, ref))
+    torch.cuda.synchronize()
+    outs = []
+    for rep in range(2):
+        for t, host, _ in cases:
+            o = torch.empty((w.batch, w.seqlen, w.dim), dtype=torch.bfloat16, pin_memory=True)
+            scan.selective_scan_fwd_host(host["u"], host["delta"], t["A"], host["B"], host["C"],
+                                         D=t["D"], z=host["z"], delta_bias=t["delta_bias"],
+                                         out=o, chunks=4)
+            outs.append(o)
+    torch.cuda.synchronize()
+    for i, o in enumerate(outs):
+        assert torch.equal(o, cases[i % len(cases)][2].cpu()), i
+
+
 def test_host_buffers_directions_inputs_and_conv(cuda_device):
     w = wl.variant("cromb", name="host_c", batch=3, seqlen=150, dim=32, conv=4, seed=172)
     _host_case(wl.make_inputs(w), cuda_device, chunks=2)
