@@ -201,3 +201,24 @@ def test_index_map_large_L():
         assert scan.ss_direction_position(None, 0, L, t) == t
         dm = scan.make_dirmap((1,))
         assert scan.ss_direction_position(dm, 0, L, t) == L - 1 - t
+
+
+def test_host_buffer_call_checks_arguments_before_any_cuda_call():
+    # selective_scan_fwd_host validates every argument once, up front: shapes and dtypes of the
+    # host tensors first, then that the parameters are device tensors
+    import torch
+    dev = torch.device("cuda", 0)
+    b, L, D, N = 2, 48, 16, 4
+    u = torch.zeros((b, L, D), dtype=torch.bfloat16)
+    delta = torch.zeros((1, b, L, D), dtype=torch.bfloat16)
+    B = torch.zeros((1, b, L, N), dtype=torch.bfloat16)
+    C = torch.zeros((1, b, L, N), dtype=torch.bfloat16)
+    A = torch.zeros((D, N), dtype=torch.float32)  # not on the device
+    with pytest.raises(ValueError, match="delta"):
+        scan.selective_scan_fwd_host(u, delta[:, :, :-1], A, B, C, device=dev)
+    with pytest.raises(TypeError, match="B"):
+        scan.selective_scan_fwd_host(u, delta, A, B.float(), C, device=dev)
+    with pytest.raises(ValueError, match="z"):
+        scan.selective_scan_fwd_host(u, delta, A, B, C, z=u[:, 1:], device=dev)
+    with pytest.raises(ValueError, match="A must be a CUDA tensor"):
+        scan.selective_scan_fwd_host(u, delta, A, B, C, device=dev)
