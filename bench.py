@@ -10,11 +10,13 @@ once, out written once, parameters and last_state) / device time, summed over ra
 torchrun every rank runs the whole workload on its own GPU (independent problems, weak
 scaling, no collective on the data path); the step time is the max over ranks.
 
-The JSON line also carries: roofline (FP32 FLOP/s of the scan pipeline against the FP32 peak,
-with the HBM fraction and the instruction-issue fraction beside it; DRAM traffic and warp
-instructions per step come from the committed ncu record while the kernel sources match it),
-e2e (the public host-buffer call selective_scan_fwd_host, copies included), clocks (NVML during
-the timed region), gpu_launches and cpu_baseline (the oracle on the host cores).
+The JSON line also carries: roofline (the HBM roofline of the scan pipeline: algorithmic bytes
+over the pipeline's event time against the measured copy bandwidth; beside it the FP32, MUFU and
+instruction-issue fractions against ceilings measured live by the probes of libss_probe.so; DRAM
+traffic and warp instructions per step come from the committed ncu record while the kernel
+sources match it), e2e (the C entry point selective_scan_fwd_host from pinned host buffers to
+pinned host buffers, copies included), clocks (NVML during the timed region), gpu_launches and
+cpu_baseline (the oracle on the host cores).
 
 --impl reference runs the fp64 CPU oracle on a bounded sample of the same workload on the host
 cores (there is no other implementation of this path to compare with).
@@ -41,12 +43,16 @@ from selective_state_space_13_b200 import workloads as wl  # noqa: E402
 
 METRIC = "selective-scan achieved HBM GB/s and % of peak; state-updates/s at 1 B200"
 UNIT = "GB/s"
-DEFAULT_WORKLOAD = "m130"
+DEFAULT_WORKLOAD = "long"
 FALLBACK_HBM_GBS = 6650.0
 FLUSH_BYTES = 256 << 20
-# FP32 work of one state update in the form the kernels compute (the exp(Delta*A) of a state
-# taken as one multiply of the power chain, the state multiply-add, the readout multiply-add)
-FLOP_PER_UPDATE = 5
+# FP32 operations of one state update in the form the kernels compute: the power-chain multiply
+# that gives exp(Delta*A[d,n]), the state multiply-add and the readout multiply-add
+FP32_OPS_PER_UPDATE = 3
+# MUFU operations per step and channel: ex2 and lg2 of the softplus, ex2 of exp(Delta*A[d,0]),
+# the reciprocal of the normalisation, and tanh of the silu gate (with z)
+MUFU_PER_STEP = 4
+MUFU_PER_STEP_GATE = 5
 CPU_SECONDS = 10.0  # CPU work the cpu_baseline sample runs (repeating a small sample)
 # workloads whose description states that last_state is returned
 RETURNS_LAST_STATE = {"tiny", "long"}
@@ -151,7 +157,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.002):
+    def __init__(self, index: int, period_s: float = 0.0005):
         self.index, self.period = index, period_s
         self.samples, self.reasons = [], set()
         self.max_mhz = None
@@ -223,6 +229,34 @@ def workload_bytes(w: wl.Workload) -> int:
     return w.algorithmic_bytes(with_last_state=w.name in RETURNS_LAST_STATE)
 
 
+def config_of(w: wl.Workload, args, world: int) -> dict:
+    """The workload description both arms print (identical keys and values)."""
+    return {"workload": describe(w) + (" (seqlen overridden to %d)" % w.seqlen if args.seqlen else ""),
+            "name": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
+            "dstate": w.dstate, "directions": w.K, "gate": w.gate,
+            "returns_last_state": w.name in RETURNS_LAST_STATE, "conv": w.conv,
+            "delta_int8": w.delta_int8,
+            "parallelism": ("%d ranks, one workload each" % world) if world > 1 else "1 GPU",
+            "l2": "flushed (256 MiB write) before every timed step"}
+
+
+def probe_ceilings() -> dict:
+    """FP32, MUFU and issue ceilings measured on this GPU by the probes of libss_probe.so."""
+    import ctypes
+    from selective_state_space_13_b200 import build as b
+    lib = ctypes.CDLL(b.build_probe())
+    out = {}
+    for name in ("ffma2", "ffma", "ex2", "issue"):
+        fn = getattr(lib, "ss_probe_" + name)
+        fn.restype = ctypes.c_int
+        fn.argtypes = [ctypes.POINTER(ctypes.c_double)]
+        v = ctypes.c_double(0.0)
+        if fn(ctypes.byref(v)) != 0:
+            raise RuntimeError("probe %s failed" % name)
+        out[name] = v.value
+    return out
+
+
 # ----------------------------------------------------------------------------- CPU baseline
 
 def oracle_sample_plan(w: wl.Workload, target_updates: float):
@@ -274,8 +308,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded, %s)" % describe(w),
-            "config": {"workload": describe(w), "name": w.name, "conv": w.conv,
-                       "delta_int8": w.delta_int8},
+            "config": config_of(w, args, world),
             "updates_per_s": w.updates() * frac / step_s,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": sample},
@@ -369,12 +402,8 @@ def run_ours(args):
     updates_s = world * w.updates() / (step_ms * 1e-3)
     peak, peak_src, peaks = load_peaks()
     achieved = nbytes / (kern_ms * 1e-3) / 1e9
-    # ALU roofline: FP32 FLOPs the method needs per state update, over the FP32 peak derived
-    # from B200's unit counts and the clock (148 SMs x 128 FP32 lanes x 2 FLOP per FMA)
-    sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
-    fp32_peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
-    flops = FLOP_PER_UPDATE * w.updates()
-    alu_achieved = flops / (kern_ms * 1e-3) / 1e12
+    # the FP32, MUFU and issue ceilings of this GPU, measured now (libss_probe.so)
+    ceil = probe_ceilings()
 
     # ---- end to end: pinned host inputs -> device, scan, out -> pinned host, every step
     e2e = None
@@ -392,8 +421,8 @@ def run_ours(args):
         eb = [torch.cuda.Event(enable_timing=True) for _ in range(n_e2e)]
 
         def e2e_step():
-            # the public host-buffer call: pinned host inputs in, host outputs back, with the
-            # copies and the scan of successive pieces overlapped on three streams
+            # the C entry point selective_scan_fwd_host: pinned host inputs in, host outputs
+            # back, the copies and the scans of successive pieces pipelined by the library
             scan.selective_scan_fwd_host(
                 host["u"], host["delta"], t["A"], host["B"], host["C"], D=t["D"], z=host["z"],
                 delta_bias=t["delta_bias"], softplus=w.softplus, dirs=w.dirs, H=w.H, W=w.W,
@@ -413,8 +442,9 @@ def run_ours(args):
         e2e = {"value": world * nbytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                "ms_per_step": e2e_ms, "steps": n_e2e,
-               "path": "selective_scan_fwd_host: pinned host inputs -> device, scan, device -> "
-                       "pinned host, in %d pieces overlapped on 3 streams" % args.e2e_pieces}
+               "path": "C entry point selective_scan_fwd_host: pinned host inputs -> device, "
+                       "scan, device -> pinned host, %d pieces pipelined on the library's three "
+                       "streams" % args.e2e_pieces}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0 at N = 1 only)
     cpu = None
@@ -440,48 +470,46 @@ def run_ours(args):
     counters = {} if args.seqlen else recorded_counters(
         w.name + ("_conv%d" % w.conv if w.conv else "") + ("_int8" if w.delta_int8 else ""))
     traffic = counters.get("dram_bytes_per_launch")
-    # instruction issue: the kernels are bound by it (see the counters summaries); achieved =
-    # the recorded warp instructions of one pass over the live pass time, against one warp
-    # instruction per clock on each of the 148 x 4 schedulers
-    issue = None
+    # beside the HBM roofline: the scan pipeline's FP32 work (3 operations per state update),
+    # MUFU work (per step and channel) and, from the committed ncu record, its warp instructions,
+    # each against the ceiling the probes measured on this GPU just now
+    fp32_ach = FP32_OPS_PER_UPDATE * w.updates() / (kern_ms * 1e-3)
+    mufu_ops = (MUFU_PER_STEP_GATE if w.gate and w.K == 1 else MUFU_PER_STEP) * w.updates() / w.dstate
+    mufu_ach = mufu_ops / (kern_ms * 1e-3)
+    alu = {"fp32": {"achieved": fp32_ach / 1e12, "peak": ceil["ffma2"] / 1e12,
+                    "unit": "T fp32 lane-ops/s", "frac": fp32_ach / ceil["ffma2"],
+                    "ops_per_update": FP32_OPS_PER_UPDATE,
+                    "peak_source": "measured: packed fma.rn.f32x2 probe (scalar fma: %.1f T/s)"
+                                   % (ceil["ffma"] / 1e12)},
+           "mufu": {"achieved": mufu_ach / 1e12, "peak": ceil["ex2"] / 1e12,
+                    "unit": "T MUFU ops/s", "frac": mufu_ach / ceil["ex2"],
+                    "ops_per_step_and_channel": mufu_ops / (w.updates() / w.dstate),
+                    "peak_source": "measured: ex2.approx probe"}}
     if counters.get("warp_instructions_per_launch"):
-        issue_peak = 148 * 4 * sm_mhz * 1e6 / 1e12
-        issue_ach = counters["warp_instructions_per_launch"] / (kern_ms * 1e-3) / 1e12
-        issue = {"achieved": issue_ach, "peak": issue_peak, "unit": "T warp-instructions/s",
-                 "frac": issue_ach / issue_peak,
-                 "warp_instructions_per_launch": counters["warp_instructions_per_launch"],
-                 "source": "ncu smsp__inst_executed.sum, profiles/traffic.json"}
+        issue_ach = counters["warp_instructions_per_launch"] / (kern_ms * 1e-3)
+        alu["issue"] = {"achieved": issue_ach / 1e12, "peak": ceil["issue"] / 1e12,
+                        "unit": "T warp-instructions/s", "frac": issue_ach / ceil["issue"],
+                        "warp_instructions_per_launch": counters["warp_instructions_per_launch"],
+                        "peak_source": "measured: fp32 + integer issue probe; instructions from "
+                                       "ncu smsp__inst_executed.sum (profiles/traffic.json)"}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == wl.BF16 else "f32",
         "data": "synthetic (seeded N(0,1) inputs, A=-(n+1), log-uniform Delta bias)",
-        "config": {"workload": describe(w) + (
-                       " (seqlen overridden to %d)" % w.seqlen if args.seqlen else ""),
-                   "name": w.name, "batch": w.batch,
-                   "seqlen": w.seqlen, "dim": w.dim, "dstate": w.dstate, "directions": w.K,
-                   "gate": w.gate, "returns_last_state": want_last, "conv": w.conv,
-                   "delta_int8": w.delta_int8,
-                   "parallelism": "independent problems per rank" if world > 1 else "1 GPU",
-                   "l2": "flushed (256 MiB write) before every timed step",
-                   "segments": args.segments or "auto", "workspace_bytes": ws_bytes},
+        "config": config_of(w, args, world),
+        "plan": {"segments": args.segments or "auto", "workspace_bytes": ws_bytes},
         "hbm_frac_of_peak": value / world / peak,
         "updates_per_s": updates_s,
-        "roofline": {"bound": "alu",
-                     "kernel": "scan pipeline: scan_kernel launches (segment aggregates, if any, "
-                               "and the scan; the direction merge excluded)",
-                     "achieved": alu_achieved, "peak": fp32_peak, "unit": "TFLOP/s",
-                     "frac": alu_achieved / fp32_peak, "traffic": traffic,
-                     "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x %.0f MHz "
-                                    "(no measured FP32 figure in MEASURED_PEAKS.json)" % sm_mhz,
-                     "algorithmic_flop_per_launch": flops,
-                     "flop_per_update": FLOP_PER_UPDATE,
-                     "kernel_ms": kern_ms,
-                     "hbm": {"achieved": achieved, "peak": peak, "unit": "GB/s",
-                             "frac": achieved / peak, "peak_source": peak_src,
-                             "algorithmic_bytes_per_launch": nbytes},
-                     "issue": issue},
+        "roofline": {"bound": "hbm",
+                     "kernel": "scan pipeline: the segment-aggregate launch (if any) and the scan "
+                               "launch, timed with CUDA events the library records around them "
+                               "(the direction merge excluded)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "peak_source": peak_src,
+                     "algorithmic_bytes_per_launch": nbytes, "kernel_ms": kern_ms,
+                     "alu": alu},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": sampler.report(),
         "e2e": e2e,

@@ -37,15 +37,22 @@
  *     `workspace` buffer, sized by selective_scan_workspace_size().
  *   - Work is enqueued on `stream` (a cudaStream_t, passed as void*; NULL = legacy default
  *     stream).  No call synchronises the stream except selective_scan_device_status().
- *   - Arguments are validated before anything is launched.  On any error status nothing has
- *     been launched and no memory has been read or written.
+ *   - Arguments are validated, tensor maps encoded and kernel attributes set before anything is
+ *     launched: on any error status other than SS_ERR_CUDA nothing has been launched and no
+ *     memory has been read or written.  SS_ERR_CUDA means the runtime failed; when it failed
+ *     at a later launch of a call (the scan after the segment aggregates, or the direction
+ *     merge), the earlier launches of that call have been enqueued.
+ *   - `stream` must belong to the current device (SS_ERR_DEVICE otherwise): the library's
+ *     device-side words are looked up on the current device.
  *   - Base pointers of u, delta, B, C, z, out and workspace must be 16-byte aligned, and
  *     dim * sizeof(io element) must be a multiple of 16 (SS_ERR_ALIGN otherwise).
  *   - N (dstate) is at most SS_MAX_DSTATE; at most SS_MAX_DIRS directions.
  *   - There is no CPU fallback: without a CUDA device every launch returns SS_ERR_CUDA.
  *   - The first selective_scan_fwd call on each device looks up the address of the library's
  *     device error word (cudaGetSymbolAddress, once); make that first call before capturing a
- *     stream into a CUDA graph.
+ *     stream into a CUDA graph.  The cached address (and the no-allocation scratch address of
+ *     selective_scan_fwd_noalloc) belongs to the device's current context: after a
+ *     cudaDeviceReset the library must not be called again in the same process.
  */
 #ifndef SELECTIVE_SCAN_H
 #define SELECTIVE_SCAN_H
@@ -57,7 +64,7 @@
 extern "C" {
 #endif
 
-#define SS_ABI_VERSION 4
+#define SS_ABI_VERSION 5
 #define SS_MAX_DSTATE 16
 #define SS_MAX_DIRS 4
 #define SS_MAX_CONV_WIDTH 4
@@ -73,8 +80,9 @@ typedef enum {
     SS_ERR_CUDA = 7,          /* the CUDA runtime reported an error at launch                  */
     SS_ERR_WORKSPACE = 8,     /* workspace NULL or smaller than selective_scan_workspace_size  */
     SS_ERR_DEVICE_TIMEOUT = 9, /* a kernel gave up a bounded wait (reported by device_status)  */
-    SS_ERR_SCRATCH_LIMIT = 10  /* selective_scan_fwd_noalloc: the problem needs more scratch than
+    SS_ERR_SCRATCH_LIMIT = 10, /* selective_scan_fwd_noalloc: the problem needs more scratch than
                                   SS_NOALLOC_SCRATCH_BYTES                                      */
+    SS_ERR_DEVICE = 11         /* `stream` belongs to another device than the current one       */
 } ss_status;
 
 typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_dtype;
@@ -237,6 +245,57 @@ ss_status selective_scan_fwd_noalloc(const ss_shape* shape, const void* u, const
                                      const float* Dskip, const void* z, const float* delta_bias,
                                      int32_t softplus, const ss_direction_map* dmap, void* out,
                                      float* last_state, void* stream, const ss_launch_opts* opts);
+
+/* Pieces at most that selective_scan_fwd_host cuts a call into. */
+#define SS_HOST_MAX_PIECES 64
+
+/* Bytes of device workspace selective_scan_fwd_host needs for this problem, these options and
+ * this number of pieces (0 when the problem is empty): two staging slots of the largest piece
+ * (its u, delta, B, C, z, out, final state and, with an initial state, a copy of its slice)
+ * and the workspace of that piece's scan.  Validates like selective_scan_workspace_size;
+ * SS_ERR_UNSUPPORTED for pieces outside 1..SS_HOST_MAX_PIECES.  Host-only. */
+ss_status selective_scan_host_workspace_size(const ss_shape* shape, const ss_direction_map* dmap,
+                                             const ss_launch_opts* opts, int32_t pieces,
+                                             size_t* bytes);
+
+/*
+ * selective_scan_fwd_host -- the scan of selective_scan_fwd for activations held in HOST
+ * memory, with the results written back to host memory: one call from host buffers to host
+ * buffers, as a serving process that receives requests on the host makes it.
+ *
+ *   u, delta, B, C, z     HOST pointers, shapes and dtypes of selective_scan_fwd (z may be NULL);
+ *                         page-locked memory (cudaHostAlloc / cudaHostRegister) lets the copies
+ *                         run asynchronously; pageable memory works, but each copy then blocks
+ *                         the calling thread
+ *   out, last_state       HOST pointers (last_state may be NULL)
+ *   A, Dskip, delta_bias  DEVICE pointers: the parameters stay resident on the GPU, as do
+ *                         every device pointer of `opts` (initial_state, conv_weight,
+ *                         conv_bias, delta_scale)
+ *   workspace             DEVICE memory of selective_scan_host_workspace_size() bytes, 256-byte
+ *                         aligned; its contents on entry do not matter
+ *   pieces                1..SS_HOST_MAX_PIECES: the call is cut into this many pieces (groups
+ *                         of batch rows; for one forward direction without convolution and with
+ *                         fewer batch rows than pieces, stretches of each row's sequence of whole
+ *                         16-step tiles, each continuing from the previous one's final state)
+ *   stream                the caller's stream (of the current device)
+ *
+ * The call enqueues, on three streams of the library (created on the first call on a device and
+ * kept until exit), the host->device copies of each piece (one cudaMemcpyAsync per contiguous
+ * block), its scan (one selective_scan_fwd call on the piece) and the device->host copies of its
+ * results, pipelined so that the copies in of piece i, the scan of piece i-1 and the copies out
+ * of piece i-2 overlap.  All of it is ordered after the work already enqueued on `stream`, and
+ * `stream` continues only after all of it: synchronise `stream` before reading out and
+ * last_state.  Calls on one device are serialised on the library's streams; calls from several
+ * host threads are safe.  Errors as selective_scan_fwd; SS_ERR_CUDA or a scan error from a later
+ * piece leaves the earlier pieces enqueued.  The pages have no counterpart to this entry point:
+ * it moves data; every step of the scan is selective_scan_fwd's.
+ */
+ss_status selective_scan_fwd_host(const ss_shape* shape, const void* u, const void* delta,
+                                  const float* A, const void* B, const void* C, const float* Dskip,
+                                  const void* z, const float* delta_bias, int32_t softplus,
+                                  const ss_direction_map* dmap, void* out, float* last_state,
+                                  void* workspace, size_t workspace_bytes, int32_t pieces,
+                                  void* stream, const ss_launch_opts* opts);
 
 /* Human-readable name of a status code (static storage). */
 const char* ss_status_str(ss_status status);

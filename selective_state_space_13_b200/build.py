@@ -16,6 +16,8 @@ from concurrent.futures import ThreadPoolExecutor
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libss_b200.so")
+PROBE_LIB = os.path.join(PKG, "libss_probe.so")  # pipe-throughput probes of the benchmark
+PROBE_SOURCES = sorted(glob.glob(os.path.join(PKG, "csrc", "probe", "*.cu")))
 SOURCES = sorted(glob.glob(os.path.join(PKG, "csrc", "*.cu")))
 HEADERS = sorted(glob.glob(os.path.join(PKG, "csrc", "*.h")) +
                  glob.glob(os.path.join(PKG, "csrc", "*.cuh")) +
@@ -70,5 +72,20 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def build_probe(force: bool = False) -> str:
+    """Compile the pipe-throughput probes (measurement only) into libss_probe.so."""
+    if not force and os.path.exists(PROBE_LIB) and all(
+            os.path.getmtime(f) <= os.path.getmtime(PROBE_LIB) for f in PROBE_SOURCES):
+        return PROBE_LIB
+    tmp = PROBE_LIB + ".tmp%d" % os.getpid()
+    cmd = [_nvcc()] + NVCC_FLAGS + ["-shared", "-o", tmp] + PROBE_SOURCES
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError("nvcc failed on the probes:\n" + res.stdout + res.stderr)
+    os.replace(tmp, PROBE_LIB)
+    return PROBE_LIB
+
+
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose=True))
+    print(build_probe(force="--force" in sys.argv))

@@ -10,16 +10,15 @@
 namespace {
 
 constexpr int64_t kMaxSeqlen = (int64_t{1} << 31) - 1;
-// Automatic segment choice (measured on B200): when the (direction, batch row, channel tile)
-// units give fewer than about 1.5 CTAs per SM, split each sequence into S segments so that the
-// scan launch's units * S CTAs fill one wave of the kWaveCtas resident slots (6 CTAs on each
-// of the 148 SMs) as closely as possible without starting a second, mostly idle wave; when the
-// segments would still exceed kLongSegSteps steps, S is multiplied up to whole waves again.
-// Segments never go below kMinSegSteps steps.  (With more units the segment-aggregate launch
-// costs more than the parallelism it adds.)  Measured: m130 -> 4, long -> 22, cromb -> 18,
-// 10-15% faster than a fixed target for the last two.
-constexpr int64_t kSplitBelowCtas = 222;
-constexpr int64_t kWaveCtas = 6 * 148;
+// Automatic segment choice.  A sequence is split into S segments when its (direction, batch
+// row, channel tile) units alone would leave the GPU under-occupied: fewer units than a quarter
+// of the resident CTA slots (resident CTAs per SM x 148 SMs) for the precise kernel, fewer than
+// half for the fast kernel, whose CTAs are single warps.  S is then the most segments whose
+// units * S CTAs still fit one wave of the slots, multiplied up to whole waves when segments
+// would exceed kLongSegSteps steps, and never below kMinSegSteps steps per segment.  The slot
+// count is that of B200 (148 SMs), so that the plan (and the workspace size) never depends on
+// the device present.
+constexpr int64_t kSms = 148;
 constexpr int64_t kLongSegSteps = 8192;
 constexpr int64_t kMinSegSteps = 16 * ss::kTile;
 constexpr int kMaxSegments = 1024;
@@ -150,11 +149,15 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
     if (L == 0) {
         seg = 1;
     } else if (seg == 0) {
+        const bool zoh = (pl->flags & SS_FLAG_ZOH_EXACT) != 0;
+        const bool fastk = ss::uses_fast_kernel(pl->io, zoh);
         const int64_t ctas = ((pl->D + ss::channels_per_cta() - 1) / ss::channels_per_cta()) *
                              pl->batch * pl->K;
+        const int64_t slots = ss::resident_ctas_per_sm(pl->io, zoh) * kSms;
+        const int64_t split_below = fastk ? slots / 2 : slots / 4;
         seg = 1;
-        if (ctas > 0 && ctas < kSplitBelowCtas) {
-            int64_t want = kWaveCtas / ctas;  // >= 4: ctas < kSplitBelowCtas
+        if (ctas > 0 && ctas < split_below) {
+            int64_t want = slots / ctas;  // >= 2
             const int64_t waves = (L + want * kLongSegSteps - 1) / (want * kLongSegSteps);
             if (waves > 1)
                 want *= waves;
@@ -244,9 +247,18 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
         return SS_ERR_WORKSPACE;
 
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    // the stream must belong to the current device, whose error word the kernels report to
+    auto stream_on_current_device = [&]() -> ss_status {
+        int dev = 0, sdev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaStreamGetDevice(strm, &sdev) != cudaSuccess)
+            return SS_ERR_CUDA;
+        return sdev == dev ? SS_OK : SS_ERR_DEVICE;
+    };
     if (!has_data) {
         // no step is taken: the final state is the initial state (zero when none is given)
         if (last_state && has_state && pl.L == 0) {
+            if ((st = stream_on_current_device()) != SS_OK)
+                return st;
             const size_t n = static_cast<size_t>(pl.K) * pl.batch * pl.D * pl.N * sizeof(float);
             const cudaError_t e =
                 pl.init_state
@@ -258,6 +270,8 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
         return SS_OK;
     }
 
+    if ((st = stream_on_current_device()) != SS_OK)
+        return st;
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     ss::ScanParams p;
     std::memset(&p, 0, sizeof(p));
@@ -300,6 +314,9 @@ ss_status selective_scan_fwd(const ss_shape* shape, const void* u, const void* d
     p.conv_width = pl.conv_width;
     p.delta_scale = pl.delta_scale;
 
+    // tensor maps and kernel attributes for every launch of the call, before the first one
+    if (ss::prepare_scan(p, pl.io) != cudaSuccess)
+        return SS_ERR_CUDA;
     // the timing events bracket the scan pipeline: the segment-aggregate launch (if any) and
     // the scan launch, which may overlap (nothing is recorded between them)
     if (pl.ev_begin && cudaEventRecord(pl.ev_begin, strm) != cudaSuccess)
@@ -364,6 +381,8 @@ const char* ss_status_str(ss_status status)
     case SS_ERR_DEVICE_TIMEOUT: return "SS_ERR_DEVICE_TIMEOUT: a kernel gave up a bounded wait";
     case SS_ERR_SCRATCH_LIMIT:
         return "SS_ERR_SCRATCH_LIMIT: the problem needs more scratch than SS_NOALLOC_SCRATCH_BYTES";
+    case SS_ERR_DEVICE:
+        return "SS_ERR_DEVICE: the stream belongs to another device than the current one";
     }
     return "unknown ss_status";
 }

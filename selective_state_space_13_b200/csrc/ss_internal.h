@@ -22,6 +22,7 @@ struct ScanParams {
     CUtensorMap tm_u, tm_z;    // u, z as [batch*L rows, D]: boxes of kTile rows x DC channels
     CUtensorMap tm_dl;         // delta as [K*batch*L rows, D], same boxes
     CUtensorMap tm_u3, tm_z3;  // u, z as [batch*H, W, D]: boxes of 8 image rows of one column
+    CUtensorMap tm_out;        // out as [batch*L rows, D] (one direction): tensor stores of tiles
     const void* u;          // [batch, L, D] io, spatial order ([K, batch, L, D] with u_per_dir)
     const void* delta;      // [K, batch, L, D] io (or int8 codes), scan order
     const float* A;         // [D, N] ([K, D, N] with params_per_dir)
@@ -64,20 +65,40 @@ struct MergeParams {
     int32_t K;
 };
 
-// Channels handled by one CTA of the scan kernel (one thread per channel).
+// Channels handled by one CTA of either scan kernel.
 int channels_per_cta();
 
 // Device address of the library's error word on the current device (looked up once per device),
 // or null if the runtime fails.
 unsigned int* status_word();
 
-// The scan launches of one io type (one translation unit each).
-cudaError_t launch_scan_f32(const ScanParams& p, int phase1, cudaStream_t stream);
-cudaError_t launch_scan_bf16(const ScanParams& p, int phase1, cudaStream_t stream);
-cudaError_t launch_scan_bf16_i8(const ScanParams& p, int phase1, cudaStream_t stream);
+// The scan launches, one translation unit each: the fast kernel (bfloat16 io, delta as bfloat16
+// or int8 codes) and the precise kernel (fp32 io, or the exact ZOH).  phase1 = 1: segment
+// aggregates only (segments 0..S-2); phase1 = 0: the scan of all S segments.  With
+// prepare_only nothing is launched: only the kernel's shared-memory attribute is set.
+cudaError_t fast_launch_bf16(const ScanParams& p, int phase1, cudaStream_t stream, bool prepare_only);
+cudaError_t fast_launch_bf16_i8(const ScanParams& p, int phase1, cudaStream_t stream,
+                                bool prepare_only);
+cudaError_t precise_launch_f32(const ScanParams& p, int phase1, cudaStream_t stream,
+                               bool prepare_only);
+cudaError_t precise_launch_bf16(const ScanParams& p, int phase1, cudaStream_t stream,
+                                bool prepare_only);
+cudaError_t precise_launch_bf16_i8(const ScanParams& p, int phase1, cudaStream_t stream,
+                                   bool prepare_only);
 
-// Enqueue one scan launch.  phase1 = 1: segment aggregates only (segments 0..S-2);
-// phase1 = 0: full scan of all S segments.  Returns the CUDA error of the launch.
+// Whether a call runs on the fast kernel (bfloat16 io without the exact ZOH) or the precise one.
+bool uses_fast_kernel(int io_dtype, bool zoh);
+
+// CTAs of a scan launch that one SM holds at once (the kernel's shared-memory and register
+// budget), for the automatic segment choice.
+int resident_ctas_per_sm(int io_dtype, bool zoh);
+
+// Everything a call needs before its first launch: the tensor maps of u, z and delta encoded into
+// p, and the shared-memory attributes of every kernel the call launches.  Nothing is launched,
+// so a failure here leaves the stream untouched.
+cudaError_t prepare_scan(ScanParams& p, int io_dtype);
+
+// Enqueue one scan launch (phase1 as above) with the tensor maps prepare_scan encoded.
 cudaError_t launch_scan(const ScanParams& p, int io_dtype, int phase1, cudaStream_t stream);
 
 // Enqueue the direction merge + gate: out = (sum_k ypart[k]) * silu(z).

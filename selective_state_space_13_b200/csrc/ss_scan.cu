@@ -4,6 +4,7 @@
 
 #include <mutex>
 
+#include "ss_fast.cuh"
 #include "ss_scan_kernels.cuh"
 
 namespace ss {
@@ -34,12 +35,49 @@ unsigned int* status_word()
 
 int channels_per_cta() { return 32 * kWarps; }
 
+bool uses_fast_kernel(int io_dtype, bool zoh) { return io_dtype == SS_BF16 && !zoh; }
+
+int resident_ctas_per_sm(int io_dtype, bool zoh)
+{
+    return uses_fast_kernel(io_dtype, zoh) ? fast::kMinBlocks : 6;
+}
+
+namespace {
+
+cudaError_t launch_any(const ScanParams& p, int io_dtype, int phase1, cudaStream_t stream,
+                       bool prepare_only)
+{
+    const bool zoh = p.zoh != 0;
+    if (uses_fast_kernel(io_dtype, zoh))
+        return p.delta_scale ? fast_launch_bf16_i8(p, phase1, stream, prepare_only)
+                             : fast_launch_bf16(p, phase1, stream, prepare_only);
+    if (io_dtype == SS_BF16)
+        return p.delta_scale ? precise_launch_bf16_i8(p, phase1, stream, prepare_only)
+                             : precise_launch_bf16(p, phase1, stream, prepare_only);
+    return precise_launch_f32(p, phase1, stream, prepare_only);
+}
+
+}  // namespace
+
+cudaError_t prepare_scan(ScanParams& p, int io_dtype)
+{
+    static_assert(fast::kCh == 32 * kWarps, "both kernels read tiles of the same channel width");
+    cudaError_t e;
+    if (io_dtype == SS_BF16)
+        e = p.delta_scale ? make_maps<__nv_bfloat16, int8_t>(p, p.z != nullptr, 32 * kWarps)
+                          : make_maps<__nv_bfloat16, __nv_bfloat16>(p, p.z != nullptr, 32 * kWarps);
+    else
+        e = make_maps<float, float>(p, p.z != nullptr, 32 * kWarps);
+    if (e != cudaSuccess)
+        return e;
+    if (p.S > 1 && (e = launch_any(p, io_dtype, 1, nullptr, true)) != cudaSuccess)
+        return e;
+    return launch_any(p, io_dtype, 0, nullptr, true);
+}
+
 cudaError_t launch_scan(const ScanParams& p, int io_dtype, int phase1, cudaStream_t stream)
 {
-    if (p.delta_scale)
-        return launch_scan_bf16_i8(p, phase1, stream);  // int8 delta needs bf16 io
-    return io_dtype == SS_BF16 ? launch_scan_bf16(p, phase1, stream)
-                               : launch_scan_f32(p, phase1, stream);
+    return launch_any(p, io_dtype, phase1, stream, false);
 }
 
 template <typename io_t, bool GATE>

@@ -1,12 +1,13 @@
-// Scan kernels instantiated for bf16 io with int8 Delta codes (a translation unit of its own so
-// that it compiles in parallel with the others).
+// The precise scan kernel instantiated for bfloat16 io with int8 delta codes (the exact ZOH
+// Bbar), in a translation unit of its own so that it compiles in parallel with the others.
 #include "ss_scan_kernels.cuh"
 
 namespace ss {
 
-cudaError_t launch_scan_bf16_i8(const ScanParams& p, int phase1, cudaStream_t stream)
+cudaError_t precise_launch_bf16_i8(const ScanParams& p, int phase1, cudaStream_t stream,
+                                   bool prepare_only)
 {
-    return launch_io<__nv_bfloat16, int8_t>(p, phase1, stream);
+    return launch_io<__nv_bfloat16, int8_t>(p, phase1, stream, prepare_only);
 }
 
 }  // namespace ss

@@ -1,4 +1,6 @@
-// Selective scan (S6) forward kernels for sm_100a.
+// The precise selective-scan kernel (S6 forward) for sm_100a: fp32 inputs, and the exact ZOH
+// Bbar for any io type.  (bfloat16 inputs with the first-order Bbar take the fast kernel of
+// ss_fast.cuh.)
 //
 // One thread owns one channel d of one (batch row, direction, segment) and keeps that channel's
 // N-state vector in registers for the whole segment ("Understanding Mamba from zero" sec. 5:
@@ -14,18 +16,10 @@
 // the C readout, the D skip and the silu gate -- happens in registers; each input element is
 // read from HBM once and each output element written once.
 //
-// Two algebraic rewrites keep the per-update work at three FP32 operations:
-//  * exp-power chain: when A[d,n] = (n+1) * A[d,0] for every n (checked in the kernel, per
-//    channel), exp(Delta*A[d,n]) = q^(n+1) with q = exp(Delta*A[d,0]): one MUFU ex2 per step and
-//    one multiply per state instead of one ex2 per state.
-//  * normalised state k = h / w with w = Delta*u: the update h = Abar*h + w*B becomes
-//    k = (w_prev/w)*Abar*k + B and y = w * (C . k), which drops the per-state w*B product.
-//    |w| is clamped below at 2^-64; this changes the B term of such a step by at most
-//    2^-64*|B| in absolute value.
-//  All exponentials run in base 2: x is carried as (delta+bias)*log2(e), so softplus in base 2
-//  gives Delta*log2(e) directly, exp(Delta*A) = ex2(Delta*log2(e) * A), and the missing ln 2
-//  of w = Delta*u is folded into the fp32 copy of B.  fp32 inputs (and the exact-ZOH Bbar) take
-//  a precise path instead: h = expm1(Delta*A)*h + (h + Bbar*u*B).
+// Arithmetic: h = (1 + expm1(Delta*A)) * h + Bbar*u*B, with expm1 from a Taylor polynomial near
+// zero, so Abar is never rounded to fp32 and the per-step error does not grow with the memory
+// length 1/|Delta*A|; softplus uses log1p from an atanh series.  Bbar is Delta, or
+// expm1(Delta*A)/A with the exact ZOH.
 //
 // Long sequences are split into S segments (the chunked scan of "S4 -> Mamba" sec. 2.2): a
 // first launch scans segments 0..S-2 from a zero state and stores each end state and the
@@ -41,9 +35,9 @@
 // error word (read by selective_scan_device_status), waits a bounded time for the copies this
 // CTA still has in flight, and the whole CTA returns.
 //
-// This header holds the kernels and their launch templates; ss_scan_f32.cu, ss_scan_bf16.cu and
-// ss_scan_bf16_i8.cu instantiate them per io type and delta storage (compiled in parallel), and
-// ss_scan.cu holds the host entry points.
+// This header holds the kernel, the direction merge and their launch templates; ss_scan_f32.cu,
+// ss_scan_bf16.cu and ss_scan_bf16_i8.cu instantiate them per io type and delta storage
+// (compiled in parallel), and ss_scan.cu holds the host dispatch.
 #pragma once
 
 #include <cuda.h>
@@ -55,155 +49,11 @@
 #include <type_traits>
 
 #include "ss_internal.h"
+#include "ss_device.cuh"
 
 namespace ss {
 
 namespace {
-
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kTinyW = 5.421010862427522e-20f;  // 2^-64
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
-constexpr unsigned long long kTestWaitNs = 20000000ull;     // 20 ms (test hook)
-constexpr unsigned int kStatusTimeout = 1u;
-
-// ---------------------------------------------------------------------------- PTX wrappers
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p)
-{
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void fence_mbar_init()
-{
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
-{
-    asm volatile(
-        "{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ unsigned long long global_ns()
-{
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Wait for the phase with this parity to complete, for at most limit_ns.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  unsigned long long limit_ns)
-{
-    if (mbar_try_wait(bar, parity))
-        return true;
-    const unsigned long long t0 = global_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity))
-            return true;
-        if ((it & 31u) == 0u && global_ns() - t0 > limit_ns)
-            return false;
-    }
-}
-
-// Bulk asynchronous copy global -> shared; completes `bytes` of transaction on `bar`.
-// dst, src and bytes must be multiples of 16.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// Tiled tensor copies global -> shared through a tensor map (a __grid_constant__ parameter);
-// coordinates are in elements, innermost first.
-__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, int32_t c0, int32_t c1,
-                                       uint64_t* bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_3d(void* dst, const CUtensorMap* map, int32_t c0, int32_t c1,
-                                       int32_t c2, uint64_t* bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// Programmatic dependent launch: let the next kernel in the stream start (launch_dependents);
-// wait until the previous kernel has finished and its writes are visible (wait).
-__device__ __forceinline__ void pdl_launch_dependents()
-{
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-__device__ __forceinline__ void pdl_wait()
-{
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
-__device__ __forceinline__ float ex2(float x)
-{
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ float lg2(float x)
-{
-    float y;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ float tanh_approx(float x)
-{
-    float y;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ float rcp(float x)
-{
-    float y;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 // log(1 + e) for e in [0, 1], relative error ~1e-7: 2*atanh(s) with s = e / (2 + e) <= 1/3,
 // odd series up to s^15 (truncation < 2e-9 relative).
@@ -257,23 +107,6 @@ template <> struct Io<__nv_bfloat16> {
     }
     static __device__ __forceinline__ __nv_bfloat16 st(float v) { return __float2bfloat16_rn(v); }
 };
-
-// ---------------------------------------------------------------------------- index map
-
-// Spatial position visited at step t of a scan in direction dir over L = H*W positions laid
-// out row by row.  Written independently of the oracle's version.
-__host__ __device__ __forceinline__ int64_t position(int32_t dir, int64_t L, int32_t H, int32_t W,
-                                                     int64_t t)
-{
-    if (dir == SS_DIR_FWD)
-        return t;
-    if (dir == SS_DIR_REV)
-        return L - 1 - t;
-    const int64_t s = (dir == SS_DIR_COL_REV) ? (L - 1 - t) : t;  // column-major step index
-    const int64_t col = s / H;
-    const int64_t row = s - col * H;
-    return row * W + col;
-}
 
 // ---------------------------------------------------------------------------- shared layout
 
@@ -335,10 +168,6 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     // the producer refills the stage released two tiles back and prepares the next tile, so at
     // least four stages are needed for a tile to be in flight while the current one is scanned
     static_assert(kStages >= 4, "the pipeline needs at least four stages");
-    // fp32 inputs take the precise arithmetic, bf16 inputs the fast one
-    constexpr bool PRECISE = sizeof(io_t) == 4;
-    // the precise arithmetic also serves the exact-ZOH Bbar for any io type
-    const bool precise = PRECISE || p.zoh != 0;
     constexpr int DC = Lay::DC;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
@@ -512,7 +341,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
         const io_t* br = reinterpret_cast<const io_t*>(smem + Lay::OFF_BR + st * Lay::BCRAW) + bskip;
         const io_t* cr = reinterpret_cast<const io_t*>(smem + Lay::OFF_CR + st * Lay::BCRAW) + cskip;
         float* bf = reinterpret_cast<float*>(smem + Lay::OFF_BF + st * Lay::BF_STRIDE);
-        const float bscale = precise ? 1.f : kLn2;
+        const float bscale = 1.f;
         if (NS == 16 && p.N == 16 && sizeof(io_t) == 2 && bskip == 0 && cskip == 0) {
             // 16 bf16 rows of 16 values per tensor: lane l converts 8 values (16 bytes) of B and
             // 8 of C; rows past the tile's end become 0
@@ -547,33 +376,25 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     };
 
     // ---- per-channel constants
-    float a_l[NS];       // A[d, n] (natural units; multiplies Delta*log2(e))
-    bool chain = true;   // A[d, n] == (n+1) * A[d, 0] for all n
-    float dskip = 0.f, bias2 = 0.f, bias_raw = 0.f;
-    float dscale = 1.f, dscale2 = kLog2e;  // int8 codes: scale[d], and scale[d] * log2(e)
+    float a_l[NS];       // A[d, n]
+    float dskip = 0.f, bias_raw = 0.f;
+    float dscale = 1.f;  // int8 codes: scale[d]
     if (active) {
         // parameters of this direction (one set shared by all directions unless per direction)
         const int64_t pk = p.params_per_dir ? static_cast<int64_t>(k) : 0;
         const float* Ak = p.A + pk * p.D * p.N;
 #pragma unroll
-        for (int n = 0; n < NS; ++n) {
+        for (int n = 0; n < NS; ++n)
             a_l[n] = (n < p.N) ? Ak[d * p.N + n] : 0.f;
-            if (n < p.N && a_l[n] != static_cast<float>(n + 1) * a_l[0])
-                chain = false;
-        }
         dskip = p.Dskip ? p.Dskip[pk * p.D + d] : 0.f;
         bias_raw = p.bias ? p.bias[pk * p.D + d] : 0.f;
-        bias2 = bias_raw * kLog2e;
-        if (DQ) {
+        if (DQ)
             dscale = p.delta_scale[d];
-            dscale2 = dscale * kLog2e;
-        }
     } else {
 #pragma unroll
         for (int n = 0; n < NS; ++n)
             a_l[n] = 0.f;
     }
-    const bool use_chain = __all_sync(0xffffffffu, chain) && !p.force_generic;
     const bool softplus = p.softplus != 0;
 
     // ---- causal depthwise convolution along this direction's scan order (CONV): the taps and
@@ -600,27 +421,22 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
         xm2 = halo(t_begin - 2);
         xm3 = halo(t_begin - 3);
     }
-    // u of the current step from its raw input: the convolution and SiLU with CONV, else as is.
-    // With h = c/2 (the halved taps), silu(c) = c * sigmoid(c) = h + h * tanh(h): one MUFU
-    // operation on the fast path; the precise path takes c * 1/(1 + 2^(-c log2 e)).
-    auto conv_step = [&](float xv, auto accurate_tag) {
+    // u of the current step from its raw input: the convolution and SiLU with CONV, else as is
+    // (c = 2h from the halved taps; silu(c) = c / (1 + 2^(-c log2 e))).
+    auto conv_step = [&](float xv) {
         if (!CONV)
             return xv;
         const float h = fmaf(cw[3], xv, fmaf(cw[2], xm1, fmaf(cw[1], xm2, fmaf(cw[0], xm3, cbias))));
         xm3 = xm2;
         xm2 = xm1;
         xm1 = xv;
-        if (decltype(accurate_tag)::value) {
-            const float c = h + h;
-            return c * rcp(1.f + ex2(-c * kLog2e));
-        }
-        return fmaf(h, tanh_approx(h), h);
+        const float c = h + h;
+        return c * rcp(1.f + ex2(-c * kLog2e));
     };
 
-    // ---- state, as pairs (n, n+1): the fast path keeps k = h / w_prev, the precise path h
+    // ---- state h
     float2 kst2[NS / 2];
     float* kst = reinterpret_cast<float*>(kst2);
-    float wprev = 1.f;
 #pragma unroll
     for (int j = 0; j < NS / 2; ++j)
         kst2[j] = make_float2(0.f, 0.f);
@@ -726,13 +542,13 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
             const float* bf = reinterpret_cast<const float*>(smem + Lay::OFF_BF + st * Lay::BF_STRIDE);
             const float4* B4 = reinterpret_cast<const float4*>(bf);
             const float4* C4 = reinterpret_cast<const float4*>(bf + kTile * NS);
-            if (precise) {
+            {
                 // h = (1 + expm1(Delta*A)) h + Bbar*u*B without rounding Abar to fp32, so the
                 // per-step error does not grow with the memory length 1/|Delta*A|; Bbar is Delta,
                 // or expm1(Delta*A)/A with the exact ZOH
                 for (int r = 0; r < rows; ++r) {
                     const float uv =
-                        conv_step(Io<io_t>::ld(su + (r ^ xmask) * DC + tid), std::true_type{});
+                        conv_step(Io<io_t>::ld(su + (r ^ xmask) * DC + tid));
                     const float dr = Io<dl_t>::ld(sdl + r * DC + tid);
                     const float x = DQ ? fmaf(dr, dscale, bias_raw) : dr + bias_raw;
                     const float spv = fmaxf(x, 0.f) + log1p_unit(ex2(-fabsf(x) * kLog2e));
@@ -773,141 +589,6 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
                         }
                     }
                 }
-            } else {
-                // fast path, kGroup rows at a time: first the per-step scalars of all kGroup
-                // rows, then their state updates; no branch inside a group, so the compiler can
-                // overlap consecutive rows.  A row past the tile's end leaves the state as it
-                // is: q = 1, w = the previous w (so w_prev/w = 1), and B = 0 there.
-                auto group = [&](auto chain_tag, auto full_tag, auto dirc_tag, int r0) {
-                    constexpr bool CHAIN = decltype(chain_tag)::value;
-                    constexpr bool FULL = decltype(full_tag)::value;  // all kGroup rows valid
-                    // u/z row order inside the group: +1 ascending, -1 descending (the rows of
-                    // an aligned group run linearly for every xmask), 0 = through xmask
-                    constexpr int DIRC = decltype(dirc_tag)::value;
-                    const int rowbase = r0 ^ xmask;  // u/z row of g = 0 when DIRC != 0
-                    float s_q[kGroup], s_w[kGroup], s_rr[kGroup], s_sp[kGroup], s_du[kGroup],
-                        s_g[kGroup];
-#pragma unroll
-                    for (int g = 0; g < kGroup; ++g) {
-                        const bool valid = FULL || r0 + g < rows;
-                        const int r = valid ? (r0 + g) : (rows - 1);
-                        // (a row past the end shifts the convolution window, but it only occurs
-                        // in the segment's last tile)
-                        const int ur = DIRC == 0 ? (r ^ xmask) : rowbase + DIRC * g;
-                        const float uv =
-                            conv_step(Io<io_t>::ld(su + ur * DC + tid), std::false_type{});
-                        const float dr = Io<dl_t>::ld(sdl + r * DC + tid);
-                        // x = (delta + bias) * log2(e); Delta*log2(e) = softplus in base 2 of x
-                        const float x = fmaf(dr, DQ ? dscale2 : kLog2e, bias2);
-                        const float e = ex2(-fabsf(x));              // 2^-|x| in (0, 1]
-                        const float l_big = lg2(1.f + e);
-                        // log2(1+e) for small e: e*log2(e)*(1 - e/2), rel. error < e^2/3
-                        const float l_small = e * fmaf(e, -0.5f * kLog2e, kLog2e);
-                        const float spv = fmaxf(x, 0.f) + (e < 0.00390625f ? l_small : l_big);
-                        const float sp2 = valid ? (softplus ? spv : x) : 0.f;
-                        float w = sp2 * uv;                           // = Delta*u / ln 2
-                        w = fabsf(w) < kTinyW ? kTinyW : w;
-                        s_w[g] = valid ? w : (g == 0 ? wprev : s_w[g - 1]);
-                        s_sp[g] = sp2;
-                        s_q[g] = CHAIN ? ex2(sp2 * a_l[0]) : 1.f;
-                        s_du[g] = dskip * uv;
-                        s_g[g] = 1.f;
-                        if (GATE) {
-                            // silu(z) = z * sigmoid(z) = h + h * tanh(h) with h = z/2
-                            const float hz = 0.5f * Io<io_t>::ld(sz + ur * DC + tid);
-                            s_g[g] = fmaf(hz, tanh_approx(hz), hz);
-                        }
-                    }
-#pragma unroll
-                    for (int g = 0; g < kGroup; ++g)
-                        s_rr[g] = (g == 0 ? wprev : s_w[g - 1]) * rcp(s_w[g]);
-                    wprev = s_w[kGroup - 1];
-#pragma unroll
-                    for (int g = 0; g < kGroup; ++g) {
-                        const int r = r0 + g;  // < kTile; rows past the tile end read B = C = 0
-                        const float rr = s_rr[g];
-                        if (PHASE1)
-                            dsum += s_sp[g];
-                        // c[n] = (w_prev/w) * exp(Delta*A[d,n]) as pairs (n, n+1)
-                        float2 cp[NS / 2];
-                        if (CHAIN) {
-                            // q^(n+1): pair j = pair (j-1) * (q^2, q^2); the rows of a group are
-                            // independent, so the chain's depth costs no issue slots
-                            const float q = s_q[g];
-                            const float q2 = q * q;
-                            cp[0] = make_float2(rr * q, rr * q2);
-                            const float2 qq = make_float2(q2, q2);
-#pragma unroll
-                            for (int j = 1; j < NS / 2; ++j)
-                                cp[j] = __fmul2_rn(cp[j - 1], qq);
-                        } else {
-                            const float sp2 = s_sp[g];
-#pragma unroll
-                            for (int j = 0; j < NS / 2; ++j)
-                                cp[j] = make_float2(rr * ex2(sp2 * a_l[2 * j]),
-                                                    rr * ex2(sp2 * a_l[2 * j + 1]));
-                        }
-                        // C . k in two packed accumulators (fewer adds at the end than four),
-                        // started by the products of the first four states (no zeroing)
-                        float2 yacc[2];
-#pragma unroll
-                        for (int n4 = 0; n4 < NS / 4; ++n4) {
-                            const float4 bq = B4[r * (NS / 4) + n4];
-                            kst2[2 * n4] =
-                                __ffma2_rn(cp[2 * n4], kst2[2 * n4], make_float2(bq.x, bq.y));
-                            kst2[2 * n4 + 1] = __ffma2_rn(cp[2 * n4 + 1], kst2[2 * n4 + 1],
-                                                          make_float2(bq.z, bq.w));
-                            if (!PHASE1) {
-                                const float4 cq = C4[r * (NS / 4) + n4];
-                                if (n4 == 0) {
-                                    yacc[0] = __fmul2_rn(make_float2(cq.x, cq.y), kst2[0]);
-                                    yacc[1] = __fmul2_rn(make_float2(cq.z, cq.w), kst2[1]);
-                                } else {
-                                    yacc[0] = __ffma2_rn(make_float2(cq.x, cq.y),
-                                                         kst2[2 * n4], yacc[0]);
-                                    yacc[1] = __ffma2_rn(make_float2(cq.z, cq.w),
-                                                         kst2[2 * n4 + 1], yacc[1]);
-                                }
-                            }
-                        }
-                        if (!PHASE1) {
-                            const float2 ys = __fadd2_rn(yacc[0], yacc[1]);
-                            float y = fmaf(s_w[g], ys.x + ys.y, s_du[g]);
-                            if (FULL || r < rows) {
-                                if (YPART) {
-                                    yp_out[orow[r]] = y;
-                                } else {
-                                    if (GATE)
-                                        y *= s_g[g];
-                                    o_out[orow[r]] = Io<io_t>::st(y);
-                                }
-                            }
-                        }
-                    }
-                };
-                using Up = std::integral_constant<int, 1>;
-                using Down = std::integral_constant<int, -1>;
-                using Any = std::integral_constant<int, 0>;
-                for (int r0 = 0; r0 < rows; r0 += kGroup) {
-                    const bool full_group = r0 + kGroup <= rows;  // the same for the whole CTA
-                    if (use_chain) {
-                        // full groups with a fixed row order: row offsets become constants.  The
-                        // multi-direction kernels run both orders at once and keep one copy of
-                        // the code (two hot copies measured slower there).
-                        if (full_group && !YPART) {
-                            if (xmask == 0)
-                                group(std::true_type{}, std::true_type{}, Up{}, r0);
-                            else
-                                group(std::true_type{}, std::true_type{}, Down{}, r0);
-                        } else if (full_group) {
-                            group(std::true_type{}, std::true_type{}, Any{}, r0);
-                        } else {
-                            group(std::true_type{}, std::false_type{}, Any{}, r0);
-                        }
-                    } else {
-                        group(std::false_type{}, std::false_type{}, Any{}, r0);
-                    }
-                }
             }
         }
         __syncwarp();
@@ -939,13 +620,13 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
 #pragma unroll
         for (int n = 0; n < NS; ++n)
             if (n < p.N)
-                p.carry_h[ci * p.N + n] = wprev * kst[n];
+                p.carry_h[ci * p.N + n] = kst[n];
     } else if (p.last_state && seg == p.S - 1) {
         float* ls = p.last_state + (kb * p.D + d) * p.N;
 #pragma unroll
         for (int n = 0; n < NS; ++n)
             if (n < p.N)
-                ls[n] = wprev * kst[n];
+                ls[n] = kst[n];
     }
 }
 
@@ -1013,110 +694,13 @@ __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ Merg
 
 constexpr int kWarps = 2;
 
-// Launch `kern(p)`; with `dependent`, the launch may begin before the previous kernel in the
-// stream has finished (programmatic dependent launch).
-template <typename Kern, typename P>
-cudaError_t launch_ex(Kern kern, unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
-                      bool dependent, const P& p)
-{
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = dependent ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, p);
-}
-
-// cuTensorMapEncodeTiled, looked up once through the runtime (no link-time libcuda dependency).
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
-        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-    }();
-    return fn;
-}
-
-// A row-major tensor of `rank` dims (innermost first) with element strides `pitch` bytes for
-// dims 1.., read in boxes `box`; out-of-range elements read as zero.
-template <typename T> constexpr CUtensorMapDataType map_type()
-{
-    return sizeof(T) == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8  // int8 codes, reinterpreted in the kernel
-           : sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-}
-
-bool encode(CUtensorMap* map, const void* base, CUtensorMapDataType type, int rank,
-            const cuuint64_t* dims, const cuuint64_t* pitch, const cuuint32_t* box)
-{
-    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
-    if (!fn)
-        return false;
-    const cuuint32_t unit[3] = {1, 1, 1};
-    return fn(map, type,
-              static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, pitch, box, unit,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-template <typename io_t, typename dl_t>
-cudaError_t make_maps(ScanParams& p, bool need_z)
-{
-    constexpr CUtensorMapDataType ty = map_type<io_t>();
-    constexpr CUtensorMapDataType ty_dl = map_type<dl_t>();
-    const cuuint64_t esz = sizeof(io_t);
-    const cuuint64_t D = static_cast<cuuint64_t>(p.D);
-    const cuuint32_t box2[2] = {static_cast<cuuint32_t>(32 * kWarps), static_cast<cuuint32_t>(kTile)};
-    const cuuint64_t pitch2[1] = {D * esz};
-    const cuuint64_t dims_bl[2] = {D, static_cast<cuuint64_t>(p.batch * p.L)};
-    const cuuint64_t dims_kbl[2] = {D, static_cast<cuuint64_t>(p.K * p.batch * p.L)};
-    const int64_t u_blocks = p.u_per_dir ? p.K * p.batch : p.batch;  // row blocks of u
-    const cuuint64_t dims_u[2] = {D, static_cast<cuuint64_t>(u_blocks * p.L)};
-    const cuuint64_t pitch_dl[1] = {D * sizeof(dl_t)};
-    if (!encode(&p.tm_u, p.u, ty, 2, dims_u, pitch2, box2) ||
-        !encode(&p.tm_dl, p.delta, ty_dl, 2, dims_kbl, pitch_dl, box2) ||
-        (need_z && !encode(&p.tm_z, p.z, ty, 2, dims_bl, pitch2, box2)))
-        return cudaErrorInvalidValue;
-    bool col = false;
-    for (int k = 0; k < p.K; ++k)
-        col = col || p.dirs[k] == SS_DIR_COL || p.dirs[k] == SS_DIR_COL_REV;
-    p.col3d = (col && p.H > 0 && p.H % 8 == 0) ? 1 : 0;
-    if (p.col3d) {
-        const cuuint32_t box3[3] = {static_cast<cuuint32_t>(32 * kWarps), 1, 8};
-        const cuuint64_t pitch3[2] = {D * esz, static_cast<cuuint64_t>(p.W) * D * esz};
-        const cuuint64_t dims3[3] = {D, static_cast<cuuint64_t>(p.W),
-                                     static_cast<cuuint64_t>(p.batch * p.H)};
-        const cuuint64_t dims3u[3] = {D, static_cast<cuuint64_t>(p.W),
-                                      static_cast<cuuint64_t>(u_blocks * p.H)};
-        if (!encode(&p.tm_u3, p.u, ty, 3, dims3u, pitch3, box3) ||
-            (need_z && !encode(&p.tm_z3, p.z, ty, 3, dims3, pitch3, box3)))
-            return cudaErrorInvalidValue;
-    }
-    return cudaSuccess;
-}
-
 template <typename io_t, typename dl_t, int NS, bool GATE, bool PHASE1, bool YPART, bool CONV>
-cudaError_t launch_t(const ScanParams& p0, cudaStream_t stream)
+cudaError_t launch_t(const ScanParams& p, cudaStream_t stream, bool prepare_only)
 {
     using Lay = Layout<io_t, dl_t, NS, kWarps, GATE, PHASE1, YPART ? 5 : 4>;
     auto kern = scan_kernel<io_t, dl_t, NS, kWarps, GATE, PHASE1, YPART, CONV>;
-    ScanParams p = p0;
-    cudaError_t e = make_maps<io_t, dl_t>(p, Lay::HAS_Z);
-    if (e != cudaSuccess)
-        return e;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::BYTES);
-    if (e != cudaSuccess)
-        return e;
+    if (prepare_only)
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::BYTES);
     const int64_t ntiles = (p.D + Lay::DC - 1) / Lay::DC;
     const int64_t nseg = PHASE1 ? (p.S - 1) : p.S;
     const int64_t nblocks = ntiles * nseg * p.batch * p.K;
@@ -1130,32 +714,33 @@ cudaError_t launch_t(const ScanParams& p0, cudaStream_t stream)
 }
 
 template <typename io_t, typename dl_t, int NS, bool CONV>
-cudaError_t launch_nc(const ScanParams& p, int phase1, cudaStream_t stream)
+cudaError_t launch_nc(const ScanParams& p, int phase1, cudaStream_t stream, bool prepare_only)
 {
     if (phase1)
-        return launch_t<io_t, dl_t, NS, false, true, false, CONV>(p, stream);
+        return launch_t<io_t, dl_t, NS, false, true, false, CONV>(p, stream, prepare_only);
     if (p.ypart)
-        return launch_t<io_t, dl_t, NS, false, false, true, CONV>(p, stream);
-    return p.z ? launch_t<io_t, dl_t, NS, true, false, false, CONV>(p, stream)
-               : launch_t<io_t, dl_t, NS, false, false, false, CONV>(p, stream);
+        return launch_t<io_t, dl_t, NS, false, false, true, CONV>(p, stream, prepare_only);
+    return p.z ? launch_t<io_t, dl_t, NS, true, false, false, CONV>(p, stream, prepare_only)
+               : launch_t<io_t, dl_t, NS, false, false, false, CONV>(p, stream, prepare_only);
 }
 
 template <typename io_t, typename dl_t, int NS>
-cudaError_t launch_ns(const ScanParams& p, int phase1, cudaStream_t stream)
+cudaError_t launch_ns(const ScanParams& p, int phase1, cudaStream_t stream, bool prepare_only)
 {
-    return p.conv_w ? launch_nc<io_t, dl_t, NS, true>(p, phase1, stream)
-                    : launch_nc<io_t, dl_t, NS, false>(p, phase1, stream);
+    return p.conv_w ? launch_nc<io_t, dl_t, NS, true>(p, phase1, stream, prepare_only)
+                    : launch_nc<io_t, dl_t, NS, false>(p, phase1, stream, prepare_only);
 }
 
-// All scan launches of io type io_t with delta stored as dl_t (io_t, or int8_t codes).
+// All scan launches of io type io_t with delta stored as dl_t (io_t, or int8_t codes); with
+// prepare_only, only the kernel's shared-memory attribute is set (nothing is launched).
 template <typename io_t, typename dl_t = io_t>
-cudaError_t launch_io(const ScanParams& p, int phase1, cudaStream_t stream)
+cudaError_t launch_io(const ScanParams& p, int phase1, cudaStream_t stream, bool prepare_only)
 {
     if (p.N <= 4)
-        return launch_ns<io_t, dl_t, 4>(p, phase1, stream);
+        return launch_ns<io_t, dl_t, 4>(p, phase1, stream, prepare_only);
     if (p.N <= 8)
-        return launch_ns<io_t, dl_t, 8>(p, phase1, stream);
-    return launch_ns<io_t, dl_t, 16>(p, phase1, stream);
+        return launch_ns<io_t, dl_t, 8>(p, phase1, stream, prepare_only);
+    return launch_ns<io_t, dl_t, 16>(p, phase1, stream, prepare_only);
 }
 
 }  // namespace

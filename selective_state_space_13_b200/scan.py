@@ -6,6 +6,7 @@ caller did not pass them, and calls the library on the current CUDA stream.  The
 path: without the library, or without a CUDA device, every call raises.
 
 The functions carry the C names: selective_scan_fwd, selective_scan_workspace_size,
+selective_scan_fwd_host, selective_scan_host_workspace_size, selective_scan_fwd_noalloc,
 ss_direction_position, selective_scan_device_status, ss_status_str, ss_abi_version.
 """
 
@@ -35,12 +36,16 @@ SS_MAX_CONV_WIDTH = 4
 
 STATUS_NAMES = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE",
                 4: "SS_ERR_ALIGN", 5: "SS_ERR_DIRMAP", 6: "SS_ERR_UNSUPPORTED", 7: "SS_ERR_CUDA",
-                8: "SS_ERR_WORKSPACE", 9: "SS_ERR_DEVICE_TIMEOUT", 10: "SS_ERR_SCRATCH_LIMIT"}
+                8: "SS_ERR_WORKSPACE", 9: "SS_ERR_DEVICE_TIMEOUT", 10: "SS_ERR_SCRATCH_LIMIT",
+                11: "SS_ERR_DEVICE"}
+SS_ERR_DEVICE = 11
+SS_HOST_MAX_PIECES = 64
 SS_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 EXPORTED = ("selective_scan_workspace_size", "selective_scan_fwd", "ss_direction_position",
             "selective_scan_device_status", "ss_status_str", "ss_abi_version",
-            "selective_scan_fwd_noalloc")
+            "selective_scan_fwd_noalloc", "selective_scan_host_workspace_size",
+            "selective_scan_fwd_host")
 
 
 class SsShape(ctypes.Structure):
@@ -126,6 +131,15 @@ def load():
         lib.ss_status_str.argtypes = [ctypes.c_int]
         lib.ss_abi_version.restype = i32
         lib.ss_abi_version.argtypes = []
+        lib.selective_scan_host_workspace_size.restype = ctypes.c_int
+        lib.selective_scan_host_workspace_size.argtypes = [ctypes.POINTER(SsShape),
+                                                           ctypes.POINTER(SsDirectionMap),
+                                                           ctypes.POINTER(SsLaunchOpts), i32,
+                                                           ctypes.POINTER(sz)]
+        lib.selective_scan_fwd_host.restype = ctypes.c_int
+        lib.selective_scan_fwd_host.argtypes = [ctypes.POINTER(SsShape), vp, vp, vp, vp, vp, vp, vp,
+                                                vp, i32, ctypes.POINTER(SsDirectionMap), vp, vp,
+                                                vp, sz, i32, vp, ctypes.POINTER(SsLaunchOpts)]
         lib.selective_scan_fwd_noalloc.restype = ctypes.c_int
         lib.selective_scan_fwd_noalloc.argtypes = [ctypes.POINTER(SsShape), vp, vp, vp, vp, vp, vp,
                                                    vp, vp, i32, ctypes.POINTER(SsDirectionMap), vp,
@@ -370,37 +384,6 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
 
 # ----------------------------------------------------------------------------- host buffers
 
-_host_streams = {}
-_host_staging = {}
-# per (device, slot): the event after the last scan that read the slot's staging inputs
-_host_slot_read = {}
-
-
-def _streams(device):
-    import torch
-    key = device.index
-    if key not in _host_streams:
-        _host_streams[key] = tuple(torch.cuda.Stream(device=device) for _ in range(3))
-    return _host_streams[key]
-
-
-def _slot(name, slot, shape, dtype, device):
-    """A device staging buffer of `shape`: a view of one allocation per (name, slot, dtype,
-    device), grown to the largest piece requested so far (so memory stays bounded by two pieces
-    per tensor, whatever shapes the calls use)."""
-    import torch
-    key = (name, slot, dtype, device.index)
-    n = 1
-    for e in shape:
-        n *= int(e)
-    buf = _host_staging.get(key)
-    if buf is None or buf.numel() < n:
-        buf = torch.empty(max(n, 1), dtype=dtype, device=device)
-        _host_staging[key] = buf
-        _host_slot_read.pop((device.index, slot), None)  # new memory: order after the caller
-    return buf[:n].view(tuple(shape))
-
-
 def _check_host(t, name, shape, dtype):
     if t is None:
         return
@@ -414,27 +397,44 @@ def _check_host(t, name, shape, dtype):
         raise ValueError("%s must be contiguous" % name)
 
 
+def selective_scan_host_workspace_size(shape: SsShape, dmap: SsDirectionMap | None, opts,
+                                       pieces: int) -> int:
+    n = ctypes.c_size_t(0)
+    st = load().selective_scan_host_workspace_size(
+        ctypes.byref(shape), ctypes.byref(dmap) if dmap is not None else None,
+        ctypes.byref(opts) if opts is not None else None, int(pieces), ctypes.byref(n))
+    if st != SS_OK:
+        raise ScanError(st, "selective_scan_host_workspace_size")
+    return int(n.value)
+
+
+def selective_scan_fwd_host_raw(shape: SsShape, u, delta, A, B, C, Dskip, z, delta_bias, softplus,
+                                dmap, out, last_state, workspace, workspace_bytes, pieces, stream,
+                                opts=None) -> int:
+    """selective_scan_fwd_host with integer addresses (host addresses for u, delta, B, C, z,
+    out and last_state; device addresses for the rest; 0 = NULL); returns the ss_status."""
+    return int(load().selective_scan_fwd_host(
+        ctypes.byref(shape), u or None, delta or None, A or None, B or None, C or None,
+        Dskip or None, z or None, delta_bias or None, int(bool(softplus)),
+        ctypes.byref(dmap) if dmap is not None else None, out or None, last_state or None,
+        workspace or None, int(workspace_bytes), int(pieces), stream or None,
+        ctypes.byref(opts) if opts is not None else None))
+
+
 def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                             dirs=(SS_DIR_FWD,), H=0, W=0, out=None, last_state=None,
                             return_last_state=False, flags=0, initial_state=None,
                             zoh_exact=False, conv_weight=None, conv_bias=None, delta_scale=None,
-                            chunks=8, device=None):
-    """Selective scan of inputs held in host memory, with the results written back to host memory.
+                            chunks=8, device=None, stream=None):
+    """Selective scan of inputs held in host memory, with the results written back to host
+    memory: one call of the C entry point selective_scan_fwd_host.
 
     u, delta, B, C, z (and out, last_state) are CPU tensors -- pinned, so that the copies are
     asynchronous -- with the shapes of selective_scan_fwd; A, D, delta_bias, conv_weight,
-    conv_bias, delta_scale and initial_state are parameters already on the device.  The work is
-    cut into `chunks` pieces and pipelined over three streams, so that the host->device copies of
-    one piece, the scan of the previous one and the device->host copy of the one before that run
-    at the same time (the two copy directions use both halves of the duplex host link).  Pieces
-    are groups of batch rows; a scan of one forward direction without convolution asked for more
-    pieces than it has batch rows cuts each row along the sequence instead, each piece continuing
-    from the previous piece's final state.  The arguments are checked once; each piece's scan is
-    one selective_scan_fwd call of the CUDA library.  The call returns once everything is
-    enqueued, ordered after the caller's current stream, which it rejoins at the end; only its
-    host->device copies start earlier, as soon as the previous call's scans have released the
-    device staging buffers, so that consecutive calls overlap.  The staging buffers and streams
-    are shared by all calls on a device: make those calls from one thread.
+    conv_bias, delta_scale and initial_state are parameters already on the device.  The library
+    cuts the work into `chunks` pieces and pipelines the host->device copies, the scans and the
+    device->host copies of successive pieces on its own streams, ordered after the current
+    stream, which continues once everything is done (synchronise it before reading out).
     Returns out, or (out, last_state) with return_last_state.
     """
     import torch
@@ -462,7 +462,6 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
         pshape = (K, Dm)
     if zoh_exact:
         flags = int(flags) | SS_FLAG_ZOH_EXACT
-    # ---- every argument is checked once here; the pieces below only slice
     _check_host(u, "u", tuple(u.shape[:-3]) + (batch, L, Dm), io)
     if delta.dtype == torch.int8:
         if delta_scale is None:
@@ -491,134 +490,37 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
     if out is None:
         out = torch.empty((batch, L, Dm), dtype=io, pin_memory=True)
     _check_host(out, "out", (batch, L, Dm), io)
-    want_last = return_last_state or last_state is not None
-    if want_last and last_state is None:
+    if return_last_state and last_state is None:
         last_state = torch.empty((K, batch, Dm, N), dtype=torch.float32, pin_memory=True)
     _check_host(last_state, "last_state", (K, batch, Dm, N), torch.float32)
 
-    # ---- pieces (r0, r1, a, b): batch rows r0..r1-1, steps a..b-1
-    nch = max(1, int(chunks))
-    carry = (K == 1 and int(dirs[0]) == SS_DIR_FWD and conv_weight is None and not u_per_dir
-             and L > 0 and (batch == 1 or nch > batch))
-    if carry:
-        parts = -(-nch // batch)
-        step = -(-L // parts)
-        step = -(-step // 16) * 16  # whole 16-step tiles
-        pieces = [(r, r + 1, a, min(L, a + step)) for r in range(batch) for a in range(0, L, step)]
-    else:
-        nb = max(1, min(nch, batch))
-        rstep = -(-batch // nb) if batch else 1
-        pieces = [(r, min(batch, r + rstep), 0, L) for r in range(0, batch, rstep)]
-    if L == 0 or Dm == 0:
-        pieces = []
-
-    # ---- the C structures: one direction map, a shape per distinct piece size, and the
-    # workspace of the largest piece
+    shape = make_shape(batch, L, Dm, N, io_code)
     dmap = make_dirmap(dirs, H, W)
-    shapes = {}
-    for r0, r1, a, b in pieces:
-        key = (r1 - r0, b - a)
-        if key not in shapes:
-            shapes[key] = make_shape(key[0], key[1], Dm, N, io_code)
-    p_conv_w, p_conv_b, p_scale = _ptr(conv_weight), _ptr(conv_bias), _ptr(delta_scale)
-    probe = make_opts(0, flags, None, 0, p_conv_w, p_conv_b, width, p_scale)
-    nws = max([selective_scan_workspace_size(sh, dmap, probe) for sh in shapes.values()] + [0])
-    p_A, p_D, p_bias = _ptr(A), _ptr(D), _ptr(delta_bias)
-
-    # the staging slots of every piece (allocated or grown here, before any copy is enqueued)
-    views_of, devs_of = [], []
-    for i, (r0, r1, a, b) in enumerate(pieces):
-        views = dict(u=u[..., r0:r1, a:b, :], delta=delta[:, r0:r1, a:b],
-                     B=B[:, r0:r1, a:b], C=C[:, r0:r1, a:b],
-                     z=None if z is None else z[r0:r1, a:b])
-        views_of.append(views)
-        devs_of.append({k: None if v is None else _slot(k, i % 2, v.shape, v.dtype, device)
-                        for k, v in views.items()})
-
-    cur = torch.cuda.current_stream(device)
-    s_in, s_comp, s_out = _streams(device)
-    start = torch.cuda.Event()
-    start.record(cur)
-    # The scans and the copies back follow the caller's stream.  The copies in only write the
-    # staging slots: they wait for the last scan of the previous call that read each slot, so
-    # that they overlap the end of that call (a slot whose memory is new waits for the caller).
-    for slot in range(min(2, len(pieces))):
-        ev = _host_slot_read.get((device.index, slot))
-        if ev is None:
-            s_in.wait_event(start)
-            break
-    else:
-        for slot in range(min(2, len(pieces))):
-            s_in.wait_event(_host_slot_read[(device.index, slot)])
-    for s in (s_comp, s_out):
-        s.wait_event(start)
-    with torch.cuda.stream(s_comp):
-        ws = _workspace(nws, device) if nws > 0 else None
-    p_ws, n_ws = _ptr(ws), (0 if ws is None else ws.numel())
-    h_comp = s_comp.cuda_stream
-    comp_done, out_done = [], []
-    prev_last = None
-    for i, (r0, r1, a, b) in enumerate(pieces):
-        slot = i % 2
-        rows, steps = r1 - r0, b - a
-        # the piece's views of the host tensors, and device slots of the same shapes
-        views, dev = views_of[i], devs_of[i]
-        oview = out[r0:r1, a:b]
-        with torch.cuda.stream(s_in):
-            if i >= 2:
-                s_in.wait_event(comp_done[i - 2])  # the scan of piece i-2 has read this slot
-            for k, v in views.items():
-                if v is None:
-                    continue
-                if v.dim() == 4 and not v.is_contiguous():  # [K, rows, ...]: one copy per k
-                    for kk in range(v.shape[0]):
-                        dev[k][kk].copy_(v[kk], non_blocking=True)
-                else:
-                    dev[k].copy_(v, non_blocking=True)
-            in_done = torch.cuda.Event()
-            in_done.record(s_in)
-        with torch.cuda.stream(s_comp):
-            s_comp.wait_event(in_done)
-            if i >= 2:
-                s_comp.wait_event(out_done[i - 2])  # the output slot has been copied out
-            o_dev = _slot("out", slot, oview.shape, io, device)
-            l_dev = _slot("last", slot, (K, rows, Dm, N), torch.float32, device) \
-                if (want_last or carry) else None
-            if carry and a > 0:
-                h0 = prev_last
-            elif initial_state is not None:
-                h0 = initial_state[:, r0:r1]
-                if not h0.is_contiguous():
-                    h0 = h0.contiguous()
-            else:
-                h0 = None
-            opts = make_opts(0, flags, None, _ptr(h0), p_conv_w, p_conv_b, width, p_scale)
-            st = selective_scan_fwd_raw(shapes[(rows, steps)], _ptr(dev["u"]), _ptr(dev["delta"]),
-                                        p_A, _ptr(dev["B"]), _ptr(dev["C"]), p_D, _ptr(dev["z"]),
-                                        p_bias, softplus, dmap, _ptr(o_dev), _ptr(l_dev), p_ws,
-                                        n_ws, h_comp, opts)
-            if st != SS_OK:
-                raise ScanError(st, "selective_scan_fwd")
-            prev_last = l_dev
-            done = torch.cuda.Event()
-            done.record(s_comp)
-            comp_done.append(done)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(done)
-            oview.copy_(o_dev, non_blocking=True)
-            if want_last and b == L:
-                for kk in range(K):
-                    last_state[kk, r0:r1].copy_(l_dev[kk], non_blocking=True)
-            od = torch.cuda.Event()
-            od.record(s_out)
-            out_done.append(od)
-    for i in range(max(0, len(pieces) - 2), len(pieces)):
-        _host_slot_read[(device.index, i % 2)] = comp_done[i]
-    for s in (s_in, s_comp, s_out):
-        ev = torch.cuda.Event()
-        ev.record(s)
-        cur.wait_event(ev)
-    if want_last and not pieces:
-        last_state.copy_(initial_state if initial_state is not None else
-                         torch.zeros_like(last_state))
+    opts = make_opts(0, flags, None, _ptr(initial_state), _ptr(conv_weight), _ptr(conv_bias),
+                     width, _ptr(delta_scale))
+    nws = selective_scan_host_workspace_size(shape, dmap, opts, int(chunks))
+    ws = _host_workspace(nws, device) if nws > 0 else None
+    st = selective_scan_fwd_host_raw(shape, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                     _ptr(D), _ptr(z), _ptr(delta_bias), softplus, dmap, _ptr(out),
+                                     _ptr(last_state), _ptr(ws), nws, int(chunks),
+                                     _stream_handle(stream), opts)
+    if st != SS_OK:
+        raise ScanError(st, "selective_scan_fwd_host")
     return (out, last_state) if return_last_state else out
+
+
+_host_ws = {}
+
+
+def _host_workspace(nbytes, device):
+    """The device workspace of the host-buffer call: one allocation per device, grown as needed.
+    Calls on one device are serialised on the library's streams, so they can share it as long
+    as the current stream orders a new allocation after the previous calls."""
+    import torch
+    buf = _host_ws.get(device.index)
+    if buf is None or buf.numel() < nbytes:
+        if buf is not None:
+            torch.cuda.current_stream(device).synchronize()
+        buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _host_ws[device.index] = buf
+    return buf

@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol():
     assert set(names) == set(scan.EXPORTED), names
     for name in names:
         assert hasattr(lib, name), name
-    assert scan.ss_abi_version() == 4
+    assert scan.ss_abi_version() == 5
 
 
 def test_status_strings():
@@ -222,3 +222,33 @@ def test_host_buffer_call_checks_arguments_before_any_cuda_call():
         scan.selective_scan_fwd_host(u, delta, A, B, C, z=u[:, 1:], device=dev)
     with pytest.raises(ValueError, match="A must be a CUDA tensor"):
         scan.selective_scan_fwd_host(u, delta, A, B, C, device=dev)
+
+
+def test_host_entry_point_validation():
+    # selective_scan_fwd_host and its workspace size validate like the device entry point, and
+    # check the piece count, the workspace and its alignment before any CUDA call
+    sh = _shape(batch=4, seqlen=256)
+    for bad in (0, -1, scan.SS_HOST_MAX_PIECES + 1):
+        with pytest.raises(scan.ScanError) as e:
+            scan.selective_scan_host_workspace_size(sh, None, None, bad)
+        assert e.value.status == 6
+    n1 = scan.selective_scan_host_workspace_size(sh, None, None, 1)
+    n4 = scan.selective_scan_host_workspace_size(sh, None, None, 4)
+    # two slots of the largest piece: one piece holds all rows, four pieces one row each
+    assert n1 > n4 > 0
+    assert scan.selective_scan_host_workspace_size(_shape(batch=0), None, None, 4) == 0
+    with pytest.raises(scan.ScanError) as e:
+        scan.selective_scan_host_workspace_size(_shape(dstate=17), None, None, 4)
+    assert e.value.status == 6
+
+    def call(u=FAKE, ws=FAKE, nws=None, pieces=4, A=FAKE):
+        return scan.selective_scan_fwd_host_raw(sh, u, FAKE, A, FAKE, FAKE, 0, 0, 0, 1, None, FAKE,
+                                                0, ws, n4 if nws is None else nws, pieces, 0)
+    assert call(u=0) == 1                 # a missing input
+    assert call(A=0) == 1                 # a missing parameter
+    assert call(ws=0) == 8                # no workspace
+    assert call(nws=n4 - 1) == 8          # too small
+    assert call(ws=FAKE + 16) == 4        # not 256-byte aligned
+    assert call(pieces=0) == 6
+    # well-formed: without a device the runtime fails, and says so
+    assert call() == 7

@@ -37,6 +37,63 @@ def test_tiny_workload(cuda_device):
     _check(wl.make_inputs("tiny"), cuda_device)
 
 
+# ----------------------------------------------------------------------------- zero and tiny steps
+# The bf16 kernel keeps the normalised state k = h / w with w = Delta*u and normalises a step
+# whose |w| is below 2^-64 by 2^-64 instead (which adds at most 2^-64*|B| to h).  These cases
+# put such steps -- u = 0 padding, Delta = 0, u so small that Delta*u underflows 2^-64 -- into
+# bf16 scans of one, two and four directions, with and without split sequences, and compare
+# every element with the oracle.
+
+ZERO_DIRS = {"fwd": ((wl.DIR_FORWARD,), 0, 0),
+             "fwd_rev": ((wl.DIR_FORWARD, wl.DIR_REVERSE), 0, 0),
+             "cross4": ((wl.DIR_FORWARD, wl.DIR_COLUMN, wl.DIR_REVERSE, wl.DIR_COLUMN_REVERSE), 30, 30)}
+
+
+def _zero_step_case(dirs_key, seed):
+    dirs, H, W = ZERO_DIRS[dirs_key]
+    L = H * W if H else 900
+    w = wl.Workload("zs_" + dirs_key, 4, L, 80, 16, wl.BF16, dirs=dirs, H=H, W=W, seed=seed)
+    inp = wl.make_inputs(w)
+    u = inp["u"]  # bf16 bit patterns [b, L, D]
+    u[0, :17] = 0                 # a padding run at the start
+    u[0, 400:401] = 0             # and a single padded step
+    u[1, 250:550] = 0             # 300 steps, across the segment boundaries of 3 segments
+    u[2, ::37] = 0                # scattered single steps
+    u[3] = 0                      # a whole row of padding
+    tiny = wl.f32_to_bf16_bits(np.full((20, w.dim), 1e-25, dtype=np.float32))
+    u[1, 600:620] = tiny          # Delta*u below 2^-64
+    u[2, 5:8, ::3] = tiny[:3, ::3]
+    return w, inp
+
+
+@pytest.mark.parametrize("segments", [1, 3])
+@pytest.mark.parametrize("dirs_key", sorted(ZERO_DIRS))
+def test_bf16_zero_and_tiny_input_steps(cuda_device, dirs_key, segments):
+    w, inp = _zero_step_case(dirs_key, 300 + segments)
+    _check(inp, cuda_device, segments=segments)
+
+
+@pytest.mark.parametrize("segments", [1, 3])
+@pytest.mark.parametrize("dirs_key", sorted(ZERO_DIRS))
+def test_bf16_zero_delta_steps(cuda_device, dirs_key, segments):
+    # softplus off, Delta = delta_raw + bias: bias values exact in bf16 and delta_raw = -bias at
+    # chosen steps give Delta = 0 there (h unchanged); elsewhere Delta is positive
+    dirs, H, W = ZERO_DIRS[dirs_key]
+    L = H * W if H else 900
+    w = wl.Workload("zd_" + dirs_key, 3, L, 64, 16, wl.BF16, dirs=dirs, H=H, W=W, seed=310,
+                    softplus=False)
+    inp = wl.make_inputs(w)
+    rng = np.random.default_rng(311)
+    bias = (rng.integers(1, 9, size=w.dim) / 16.0).astype(np.float32)   # exact in bf16
+    inp["delta_bias"] = bias
+    raw = rng.uniform(-bias[None, None, None, :] + 0.01, 0.3, size=inp["delta"].shape)
+    zero = [0, 1, 2, 17, 300, 301, 302, 303, 304, 305, L - 1]
+    raw[:, :, zero, :] = -bias[None, None, :]
+    raw[:, 1, 100:400, :] = -bias[None, :]                               # a long run
+    inp["delta"] = wl.f32_to_bf16_bits(raw.astype(np.float32))
+    _check(inp, cuda_device, segments=segments)
+
+
 @pytest.mark.parametrize("segments", [0, 1, 3])
 @pytest.mark.parametrize("dtype", [wl.BF16, wl.F32])
 def test_single_direction_ragged(cuda_device, dtype, segments):
