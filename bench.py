@@ -79,6 +79,7 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
 
 
 def sum_over_ranks(value: float, world: int, device=None) -> float:
+    """Sum of a float over all ranks (identity at world size 1)."""
     if world <= 1:
         return value
     import torch
@@ -236,7 +237,9 @@ def config_of(w: wl.Workload, args, world: int) -> dict:
             "dstate": w.dstate, "directions": w.K, "gate": w.gate,
             "returns_last_state": w.name in RETURNS_LAST_STATE, "conv": w.conv,
             "delta_int8": w.delta_int8,
-            "parallelism": ("%d ranks, one workload each" % world) if world > 1 else "1 GPU",
+            "parallelism": ("1 GPU" if world <= 1 else
+                            "%d ranks, one workload each" % world if args.shard == "replica" else
+                            "%d ranks, one workload split by %s" % (world, args.shard)),
             "l2": "flushed (256 MiB write) before every timed step"}
 
 
@@ -332,8 +335,21 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
-    w = workload_of(args)
-    inp = wl.make_inputs(w)
+    w_full = workload_of(args)
+    w = w_full
+    inp = wl.make_inputs(w_full)
+    shard_info = None
+    if args.shard != "replica" and world > 1:
+        # this rank scans its slice of the one workload (batch rows or channels); the slices
+        # are independent, so no data crosses between ranks
+        from selective_state_space_13_b200 import shard
+        axis, lo, hi, w = shard.shard_workload(w_full, world, rank,
+                                               None if args.shard == "auto" else args.shard)
+        if hi <= lo:
+            raise SystemExit("--shard %s leaves rank %d of %d without work; use fewer ranks"
+                             % (axis, rank, world))
+        inp = shard.shard_inputs(inp, axis, lo, hi)
+        shard_info = {"axis": axis, "lo": lo, "hi": hi}
     t = wl.to_device(inp, device)
     want_last = w.name in RETURNS_LAST_STATE
     out = torch.empty((w.batch, w.seqlen, w.dim), dtype=t["u"].dtype, device=device)
@@ -398,8 +414,11 @@ def run_ours(args):
         raise RuntimeError("device timeout during the timed region")
 
     nbytes = workload_bytes(w)
-    value = world * nbytes / (step_ms * 1e-3) / 1e9
-    updates_s = world * w.updates() / (step_ms * 1e-3)
+    # the whole job's bytes and updates: every rank's own (a replica or a slice), summed
+    job_bytes = sum_over_ranks(float(nbytes), world, device)
+    job_updates = sum_over_ranks(float(w.updates()), world, device)
+    value = job_bytes / (step_ms * 1e-3) / 1e9
+    updates_s = job_updates / (step_ms * 1e-3)
     peak, peak_src, peaks = load_peaks()
     achieved = nbytes / (kern_ms * 1e-3) / 1e9
     # the FP32, MUFU and issue ceilings of this GPU, measured now (libss_probe.so)
@@ -439,7 +458,7 @@ def run_ours(args):
         torch.cuda.synchronize(device)
         e2e_ms = sum(ea[i].elapsed_time(eb[i]) for i in range(n_e2e)) / n_e2e
         e2e_ms = max_over_ranks(e2e_ms, world, device)
-        e2e = {"value": world * nbytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+        e2e = {"value": job_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                "ms_per_step": e2e_ms, "steps": n_e2e,
                "path": "C entry point selective_scan_fwd_host: pinned host inputs -> device, "
@@ -495,11 +514,12 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
+        "scaling": "strong" if shard_info else "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == wl.BF16 else "f32",
         "data": "synthetic (seeded N(0,1) inputs, A=-(n+1), log-uniform Delta bias)",
-        "config": config_of(w, args, world),
-        "plan": {"segments": args.segments or "auto", "workspace_bytes": ws_bytes},
+        "config": config_of(w_full, args, world),
+        "plan": {"segments": args.segments or "auto", "workspace_bytes": ws_bytes,
+                 "shard": shard_info or args.shard},
         "hbm_frac_of_peak": value / world / peak,
         "updates_per_s": updates_s,
         "roofline": {"bound": "hbm",
@@ -531,6 +551,10 @@ def parse(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(wl.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--segments", type=int, default=0, help="0 = the library's choice")
+    ap.add_argument("--shard", choices=["replica", "batch", "channels", "auto"], default="replica",
+                    help="with several ranks: 'replica' = every rank scans the whole workload "
+                         "(weak scaling); 'batch' / 'channels' / 'auto' = every rank scans its "
+                         "slice of one workload (strong scaling, no collective on the data path)")
     ap.add_argument("--flags", type=int, default=0, help="SS_FLAG_* bits (1 = generic A)")
     ap.add_argument("--seqlen", type=int, default=0,
                     help="override the workload's sequence length (smaller cases for profiling)")
