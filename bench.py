@@ -345,9 +345,12 @@ def run_ours(args):
         from selective_state_space_13_b200 import shard
         axis, lo, hi, w = shard.shard_workload(w_full, world, rank,
                                                None if args.shard == "auto" else args.shard)
-        if hi <= lo:
-            raise SystemExit("--shard %s leaves rank %d of %d without work; use fewer ranks"
-                             % (axis, rank, world))
+        # every rank checks every slice, so all of them stop together (no collective waits)
+        empty = [r for r in range(world) if shard.shard_workload(w_full, world, r, axis)[2]
+                 <= shard.shard_workload(w_full, world, r, axis)[1]]
+        if empty:
+            raise SystemExit("--shard %s leaves rank(s) %s of %d without work; use fewer ranks"
+                             % (axis, empty, world))
         inp = shard.shard_inputs(inp, axis, lo, hi)
         shard_info = {"axis": axis, "lo": lo, "hi": hi}
     t = wl.to_device(inp, device)
