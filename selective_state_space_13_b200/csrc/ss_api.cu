@@ -184,11 +184,13 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
     size_t off = 0;
     pl->off_carry_h = pl->off_carry_s = pl->off_ypart = 0;
     if (pl->S > 1) {
+        // fp32 inputs carry their segment states in fp64 (the precise kernel's state type)
         const size_t cells = static_cast<size_t>(pl->K) * pl->batch * pl->S * pl->D;
+        const size_t cb = pl->io == SS_F32 ? sizeof(double) : sizeof(float);
         pl->off_carry_h = off;
-        off = align256(off + cells * pl->N * sizeof(float));
+        off = align256(off + cells * pl->N * cb);
         pl->off_carry_s = off;
-        off = align256(off + cells * sizeof(float));
+        off = align256(off + cells * cb);
     }
     if (pl->K > 1) {
         pl->off_ypart = off;

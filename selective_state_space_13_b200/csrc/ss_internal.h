@@ -38,8 +38,9 @@ struct ScanParams {
     const float* conv_w;    // [K, D, conv_width] causal conv taps per direction, or null
     const float* conv_b;    // [K, D] conv bias, or null (zero)
     const float* delta_scale;  // [D] scale of int8 delta codes, or null (delta in io type)
+    // segment carries: fp32 for bf16 io, fp64 for fp32 io (read through the kernels' state type)
     float* carry_h;         // [K, batch, S, D, N] end state of each segment scanned from zero
-    float* carry_s;         // [K, batch, S, D] sum over the segment of Delta*log2(e)
+    float* carry_s;         // [K, batch, S, D] sum over the segment of Delta (times log2(e) in fp32)
     int64_t batch, L, D;
     int64_t seg_len;        // steps per segment (last segment may be shorter)
     int32_t N, K, S;

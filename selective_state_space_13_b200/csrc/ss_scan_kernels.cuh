@@ -19,7 +19,12 @@
 // Arithmetic: h = (1 + expm1(Delta*A)) * h + Bbar*u*B, with expm1 from a Taylor polynomial near
 // zero, so Abar is never rounded to fp32 and the per-step error does not grow with the memory
 // length 1/|Delta*A|; softplus uses log1p from an atanh series.  Bbar is Delta, or
-// expm1(Delta*A)/A with the exact ZOH.
+// expm1(Delta*A)/A with the exact ZOH.  With fp32 inputs the state, the C readout and the
+// segment carries are fp64 (B200 runs fp64 at half the fp32 rate): an fp32 state loses about
+// one rounding of |h| per step, which over thousands of steps of a slowly decaying state
+// reaches the 1e-4 relative bar at near-zero outputs; in fp64 the error is that of the fp32
+// per-step factors (Delta, expm1), which does not accumulate.  bfloat16 inputs (exact ZOH) keep
+// an fp32 state.
 //
 // Long sequences are split into S segments (the chunked scan of "S4 -> Mamba" sec. 2.2): a
 // first launch scans segments 0..S-2 from a zero state and stores each end state and the
@@ -111,7 +116,7 @@ template <> struct Io<__nv_bfloat16> {
 // ---------------------------------------------------------------------------- shared layout
 
 // One pipeline stage holds kTile rows of u, delta and z for the CTA's channels (as copied),
-// the raw B and C tiles, their fp32 copies, and the output row offsets of the tile.
+// the raw B and C tiles, their copies in the state type, and the output row offsets of the tile.
 template <typename io_t, typename dl_t, int NS, int WARPS, bool GATE, bool PHASE1, int STAGES>
 struct Layout {
     static constexpr int DC = 32 * WARPS;                           // channels per CTA
@@ -128,8 +133,9 @@ struct Layout {
     static constexpr int OFF_Z = OFF_DL + STAGES * ROWS_DL;
     static constexpr int OFF_BR = OFF_Z + (HAS_Z ? STAGES * ROWS : 0);
     static constexpr int OFF_CR = OFF_BR + STAGES * BCRAW;
-    static constexpr int OFF_BF = OFF_CR + (HAS_C ? STAGES * BCRAW : 0);  // fp32 B, then fp32 C
-    static constexpr int BF_ONE = kTile * NS * 4;
+    // B, then C, converted to the state type (fp64 for fp32 io, else fp32)
+    static constexpr int OFF_BF = OFF_CR + (HAS_C ? STAGES * BCRAW : 0);
+    static constexpr int BF_ONE = kTile * NS * (std::is_same<io_t, float>::value ? 8 : 4);
     static constexpr int BF_STRIDE = BF_ONE * (HAS_C ? 2 : 1);
     static constexpr int OFF_OUT = OFF_BF + STAGES * BF_STRIDE;           // int32 row offsets
     static constexpr int OUT_STRIDE = kTile * 4;
@@ -165,6 +171,11 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     using Lay = Layout<io_t, dl_t, NS, WARPS, GATE, PHASE1, kStages>;
     // int8 Delta codes: delta_raw = code * delta_scale[d]
     constexpr bool DQ = std::is_same<dl_t, int8_t>::value;
+    // fp32 io: fp64 state, readout and carries
+    constexpr bool WIDE = std::is_same<io_t, float>::value;
+    using st_t = typename std::conditional<WIDE, double, float>::type;
+    st_t* const carry_h = reinterpret_cast<st_t*>(p.carry_h);
+    st_t* const carry_s = reinterpret_cast<st_t*>(p.carry_s);
     // the producer refills the stage released two tiles back and prepares the next tile, so at
     // least four stages are needed for a tile to be in flight while the current one is scanned
     static_assert(kStages >= 4, "the pipeline needs at least four stages");
@@ -340,15 +351,15 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
             bc_src(gC, t0, rows, bytes, cskip);
         const io_t* br = reinterpret_cast<const io_t*>(smem + Lay::OFF_BR + st * Lay::BCRAW) + bskip;
         const io_t* cr = reinterpret_cast<const io_t*>(smem + Lay::OFF_CR + st * Lay::BCRAW) + cskip;
-        float* bf = reinterpret_cast<float*>(smem + Lay::OFF_BF + st * Lay::BF_STRIDE);
+        st_t* bf = reinterpret_cast<st_t*>(smem + Lay::OFF_BF + st * Lay::BF_STRIDE);
         const float bscale = 1.f;
-        if (NS == 16 && p.N == 16 && sizeof(io_t) == 2 && bskip == 0 && cskip == 0) {
+        if (!WIDE && NS == 16 && p.N == 16 && sizeof(io_t) == 2 && bskip == 0 && cskip == 0) {
             // 16 bf16 rows of 16 values per tensor: lane l converts 8 values (16 bytes) of B and
             // 8 of C; rows past the tile's end become 0
             static_assert(kTile * 16 * 2 == 32 * 16, "one 16-byte chunk per lane and tensor");
             const int r = lane >> 1;
             const bool ok = r < rows;
-            auto cvt8 = [&](const io_t* src, float* dst, float scale) {
+            auto cvt8 = [&](const io_t* src, st_t* dst, float scale) {
                 const uint4 w = *reinterpret_cast<const uint4*>(src + 8 * lane);
                 const uint32_t v[4] = {w.x, w.y, w.z, w.w};
                 float f[8];
@@ -357,7 +368,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
                     f[2 * i] = ok ? __uint_as_float(v[i] << 16) * scale : 0.f;
                     f[2 * i + 1] = ok ? __uint_as_float(v[i] & 0xffff0000u) * scale : 0.f;
                 }
-                float4* d4 = reinterpret_cast<float4*>(dst + 8 * lane);
+                float4* d4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(dst) + 8 * lane);
                 d4[0] = make_float4(f[0], f[1], f[2], f[3]);
                 d4[1] = make_float4(f[4], f[5], f[6], f[7]);
             };
@@ -369,9 +380,9 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
         for (int idx = lane; idx < kTile * NS; idx += 32) {
             const int r = idx / NS, n = idx - (idx / NS) * NS;
             const bool ok = r < rows && n < p.N;
-            bf[idx] = ok ? Io<io_t>::ld(br + r * p.N + n) * bscale : 0.f;
+            bf[idx] = ok ? static_cast<st_t>(Io<io_t>::ld(br + r * p.N + n) * bscale) : st_t(0);
             if (Lay::HAS_C)
-                bf[kTile * NS + idx] = ok ? Io<io_t>::ld(cr + r * p.N + n) : 0.f;
+                bf[kTile * NS + idx] = ok ? static_cast<st_t>(Io<io_t>::ld(cr + r * p.N + n)) : st_t(0);
         }
     };
 
@@ -435,11 +446,10 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     };
 
     // ---- state h
-    float2 kst2[NS / 2];
-    float* kst = reinterpret_cast<float*>(kst2);
+    st_t kst[NS];
 #pragma unroll
-    for (int j = 0; j < NS / 2; ++j)
-        kst2[j] = make_float2(0.f, 0.f);
+    for (int n = 0; n < NS; ++n)
+        kst[n] = st_t(0);
     if (!PHASE1 && active && p.init_state) {
         const float* h0 = p.init_state + (kb * p.D + d) * p.N;
 #pragma unroll
@@ -455,15 +465,20 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
         // fold the carries of segments 0..seg-1: h <- exp(A * sumDelta_s) * h + h_s
         for (int s = 0; s < seg; ++s) {
             const int64_t ci = (kb * p.S + s) * p.D + d;
-            const float sd = __ldcg(p.carry_s + ci);
-            const float* ch = p.carry_h + ci * p.N;
+            const st_t sd = __ldcg(carry_s + ci);
+            const st_t* ch = carry_h + ci * p.N;
 #pragma unroll
-            for (int n = 0; n < NS; ++n)
-                if (n < p.N)
-                    kst[n] = ex2(a_l[n] * sd) * kst[n] + __ldcg(ch + n);
+            for (int n = 0; n < NS; ++n) {
+                if (n < p.N) {
+                    if (WIDE)  // sd = sum of Delta
+                        kst[n] = exp(static_cast<double>(a_l[n]) * sd) * kst[n] + __ldcg(ch + n);
+                    else       // sd = sum of Delta*log2(e)
+                        kst[n] = ex2(a_l[n] * static_cast<float>(sd)) * kst[n] + __ldcg(ch + n);
+                }
+            }
         }
     }
-    float dsum = 0.f;  // sum of Delta*log2(e) over this segment (aggregate launch)
+    st_t dsum = st_t(0);  // sum over this segment of Delta (fp64) or Delta*log2(e) (aggregate launch)
 
     // ---- pipeline.  Producer duty rotates: in iteration `it`, warp it % WARPS converts the B/C
     // of tile it+1 (one tile ahead, so no warp waits for a conversion) and refills the stage
@@ -539,7 +554,7 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
             const int32_t* orow = reinterpret_cast<const int32_t*>(smem + Lay::OFF_OUT + st * Lay::OUT_STRIDE);
             float* yp_out = p.ypart ? p.ypart + out_base + tid : nullptr;
             io_t* o_out = static_cast<io_t*>(p.out) + out_base + tid;
-            const float* bf = reinterpret_cast<const float*>(smem + Lay::OFF_BF + st * Lay::BF_STRIDE);
+            const st_t* bf = reinterpret_cast<const st_t*>(smem + Lay::OFF_BF + st * Lay::BF_STRIDE);
             const float4* B4 = reinterpret_cast<const float4*>(bf);
             const float4* C4 = reinterpret_cast<const float4*>(bf + kTile * NS);
             {
@@ -554,6 +569,37 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
                     const float spv = fmaxf(x, 0.f) + log1p_unit(ex2(-fabsf(x) * kLog2e));
                     const float dt = softplus ? spv : x;
                     const float w = dt * uv;
+                    if (WIDE) {
+                        // fp64 state and readout; the per-step factors stay fp32
+                        const double wd = static_cast<double>(dt) * static_cast<double>(uv);
+                        if (PHASE1)
+                            dsum += static_cast<double>(dt);
+                        double ypd = 0.0;
+#pragma unroll
+                        for (int n = 0; n < NS; ++n) {
+                            const float em1 = expm1_acc(dt * a_l[n]);
+                            const double wb = p.zoh && a_l[n] != 0.f
+                                                  ? static_cast<double>(em1 / a_l[n]) * static_cast<double>(uv)
+                                                  : wd;
+                            const double hb = fma(wb, static_cast<double>(bf[r * NS + n]), static_cast<double>(kst[n]));
+                            kst[n] = fma(static_cast<double>(em1), static_cast<double>(kst[n]), hb);
+                            if (!PHASE1)
+                                ypd = fma(static_cast<double>(bf[kTile * NS + r * NS + n]), static_cast<double>(kst[n]), ypd);
+                        }
+                        if (!PHASE1) {
+                            float y = static_cast<float>(fma(static_cast<double>(dskip), static_cast<double>(uv), ypd));
+                            if (YPART) {
+                                yp_out[orow[r]] = y;
+                            } else {
+                                if (GATE) {
+                                    const float zv = Io<io_t>::ld(sz + (r ^ xmask) * DC + tid);
+                                    y *= zv / (1.f + ex2(-zv * kLog2e));
+                                }
+                                o_out[orow[r]] = Io<io_t>::st(y);
+                            }
+                        }
+                        continue;
+                    }
                     if (PHASE1)
                         dsum += dt * kLog2e;
                     float yp = 0.f;
@@ -571,9 +617,9 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
                             const int n = n4 * 4 + j;
                             const float em1 = expm1_acc(dt * a_l[n]);
                             const float wb = p.zoh && a_l[n] != 0.f ? (em1 / a_l[n]) * uv : w;
-                            kst[n] = fmaf(em1, kst[n], fmaf(wb, bv[j], kst[n]));
+                            kst[n] = fmaf(em1, static_cast<float>(kst[n]), fmaf(wb, bv[j], static_cast<float>(kst[n])));
                             if (!PHASE1)
-                                yp = fmaf(cv[j], kst[n], yp);
+                                yp = fmaf(cv[j], static_cast<float>(kst[n]), yp);
                         }
                     }
                     if (!PHASE1) {
@@ -616,17 +662,17 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
         return;
     if (PHASE1) {
         const int64_t ci = (kb * p.S + seg) * p.D + d;
-        p.carry_s[ci] = dsum;
+        carry_s[ci] = dsum;
 #pragma unroll
         for (int n = 0; n < NS; ++n)
             if (n < p.N)
-                p.carry_h[ci * p.N + n] = kst[n];
+                carry_h[ci * p.N + n] = kst[n];
     } else if (p.last_state && seg == p.S - 1) {
         float* ls = p.last_state + (kb * p.D + d) * p.N;
 #pragma unroll
         for (int n = 0; n < NS; ++n)
             if (n < p.N)
-                ls[n] = kst[n];
+                ls[n] = static_cast<float>(kst[n]);
     }
 }
 
