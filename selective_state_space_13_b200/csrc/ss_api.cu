@@ -14,12 +14,13 @@ constexpr int64_t kMaxSeqlen = (int64_t{1} << 31) - 1;
 // row, channel tile) units alone would leave the GPU under-occupied: fewer units than a quarter
 // of the resident CTA slots (resident CTAs per SM x 148 SMs) for the precise kernel, fewer than
 // half for the fast kernel, whose CTAs are single warps.  S is then the most segments whose
-// units * S CTAs still fit one wave of the slots, multiplied up to whole waves when segments
-// would exceed kLongSegSteps steps, and never below kMinSegSteps steps per segment.  The slot
-// count is that of B200 (148 SMs), so that the plan (and the workspace size) never depends on
-// the device present.
+// units * S CTAs still fit one wave of the slots, and never below kMinSegSteps steps per
+// segment.  A CTA scans its whole segment, so a launch just over one wave runs a second wave of
+// whole segments (measured on B200: the long workload 4.27 ms at 14 segments, one wave of the
+// 1184 slots, against 6.02 ms at 16); and two waves double the segment carries without filling
+// the GPU better (4.47 ms at 28).  The slot count is that of B200 (148 SMs), so that the plan
+// (and the workspace size) never depends on the device present.
 constexpr int64_t kSms = 148;
-constexpr int64_t kLongSegSteps = 8192;
 constexpr int64_t kMinSegSteps = 16 * ss::kTile;
 constexpr int kMaxSegments = 1024;
 
@@ -158,9 +159,6 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
         seg = 1;
         if (ctas > 0 && ctas < split_below) {
             int64_t want = slots / ctas;  // >= 2
-            const int64_t waves = (L + want * kLongSegSteps - 1) / (want * kLongSegSteps);
-            if (waves > 1)
-                want *= waves;
             const int64_t cap = L / kMinSegSteps;
             if (want > cap)
                 want = cap;
