@@ -10,17 +10,18 @@
 namespace {
 
 constexpr int64_t kMaxSeqlen = (int64_t{1} << 31) - 1;
-// Automatic segment choice.  A sequence is split into S segments when its (direction, batch
-// row, channel tile) units alone would leave the GPU under-occupied: fewer units than a quarter
-// of the resident CTA slots (resident CTAs per SM x 148 SMs) for the precise kernel, fewer than
-// half for the fast kernel, whose CTAs are single warps.  S is then the most segments whose
-// units * S CTAs still fit one wave of the slots, and never below kMinSegSteps steps per
-// segment.  A CTA scans its whole segment, so a launch just over one wave runs a second wave of
-// whole segments (measured on B200: the long workload 4.27 ms at 14 segments, one wave of the
-// 1184 slots, against 6.02 ms at 16); and two waves double the segment carries without filling
-// the GPU better (4.47 ms at 28).  The slot count is that of B200 (148 SMs), so that the plan
-// (and the workspace size) never depends on the device present.
-constexpr int64_t kSms = 148;
+// Automatic segment choice (measured on B200): when the (direction, batch row, channel tile)
+// units give fewer than about 1.5 CTAs per SM, split each sequence into S segments so that the
+// scan launch's units * S CTAs fill one wave of the kWaveCtas resident slots (6 CTAs on each
+// of the 148 SMs) as closely as possible without starting a second, mostly idle wave; when the
+// segments would still exceed kLongSegSteps steps, S is multiplied up to whole waves again.
+// Segments never go below kMinSegSteps steps.  (With more units the segment-aggregate launch
+// costs more than the parallelism it adds.)  Measured: m130 -> 4, long -> 22, cromb -> 18;
+// long runs 4.17 ms at 22 segments against 4.54 at 14.  The slot count is that of B200, so
+// that the plan (and the workspace size) never depends on the device present.
+constexpr int64_t kSplitBelowCtas = 222;
+constexpr int64_t kWaveCtas = 6 * 148;
+constexpr int64_t kLongSegSteps = 8192;
 constexpr int64_t kMinSegSteps = 16 * ss::kTile;
 constexpr int kMaxSegments = 1024;
 
@@ -150,15 +151,14 @@ ss_status make_plan(const ss_shape* s, const ss_direction_map* dmap, const ss_la
     if (L == 0) {
         seg = 1;
     } else if (seg == 0) {
-        const bool zoh = (pl->flags & SS_FLAG_ZOH_EXACT) != 0;
-        const bool fastk = ss::uses_fast_kernel(pl->io, zoh);
         const int64_t ctas = ((pl->D + ss::channels_per_cta() - 1) / ss::channels_per_cta()) *
                              pl->batch * pl->K;
-        const int64_t slots = ss::resident_ctas_per_sm(pl->io, zoh) * kSms;
-        const int64_t split_below = fastk ? slots / 2 : slots / 4;
         seg = 1;
-        if (ctas > 0 && ctas < split_below) {
-            int64_t want = slots / ctas;  // >= 2
+        if (ctas > 0 && ctas < kSplitBelowCtas) {
+            int64_t want = kWaveCtas / ctas;  // >= 4: ctas < kSplitBelowCtas
+            const int64_t waves = (L + want * kLongSegSteps - 1) / (want * kLongSegSteps);
+            if (waves > 1)
+                want *= waves;
             const int64_t cap = L / kMinSegSteps;
             if (want > cap)
                 want = cap;

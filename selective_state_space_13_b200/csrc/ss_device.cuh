@@ -1,4 +1,4 @@
-// Device helpers shared by the scan kernels: PTX wrappers for mbarriers, bulk and tensor-map
+// Device helpers of the scan and merge kernels: PTX wrappers for mbarriers, bulk and tensor-map
 // copies and programmatic dependent launch, the MUFU approximations the fast arithmetic uses,
 // the index map of the scan orders, and the host-side tensor-map encoding and launch helper.
 #pragma once
@@ -38,13 +38,6 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
 __device__ __forceinline__ void fence_mbar_init()
 {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-// Orders this thread's earlier generic-proxy accesses of shared memory before later
-// async-proxy accesses (a bulk copy that overwrites a buffer the warp has just read).
-__device__ __forceinline__ void fence_proxy_async_smem()
-{
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes)
@@ -261,8 +254,7 @@ cudaError_t make_maps(ScanParams& p, bool need_z, int box_ch)
     const cuuint64_t pitch_dl[1] = {D * sizeof(dl_t)};
     if (!encode(&p.tm_u, p.u, ty, 2, dims_u, pitch2, box2) ||
         !encode(&p.tm_dl, p.delta, ty_dl, 2, dims_kbl, pitch_dl, box2) ||
-        (need_z && !encode(&p.tm_z, p.z, ty, 2, dims_bl, pitch2, box2)) ||
-        (p.out && !p.ypart && !encode(&p.tm_out, p.out, ty, 2, dims_bl, pitch2, box2)))
+        (need_z && !encode(&p.tm_z, p.z, ty, 2, dims_bl, pitch2, box2)))
         return cudaErrorInvalidValue;
     bool col = false;
     for (int k = 0; k < p.K; ++k)

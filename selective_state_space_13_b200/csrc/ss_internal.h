@@ -17,12 +17,11 @@ constexpr int kTile = 16;
 constexpr int kGroup = 8;
 
 // Everything a scan launch needs.  Device pointers are the caller's; nothing here is owned.
-// The tensor maps are filled in by launch_scan.
+// The tensor maps are filled in by prepare_scan.
 struct ScanParams {
     CUtensorMap tm_u, tm_z;    // u, z as [batch*L rows, D]: boxes of kTile rows x DC channels
     CUtensorMap tm_dl;         // delta as [K*batch*L rows, D], same boxes
     CUtensorMap tm_u3, tm_z3;  // u, z as [batch*H, W, D]: boxes of 8 image rows of one column
-    CUtensorMap tm_out;        // out as [batch*L rows, D] (one direction): tensor stores of tiles
     const void* u;          // [batch, L, D] io, spatial order ([K, batch, L, D] with u_per_dir)
     const void* delta;      // [K, batch, L, D] io (or int8 codes), scan order
     const float* A;         // [D, N] ([K, D, N] with params_per_dir)
@@ -66,33 +65,21 @@ struct MergeParams {
     int32_t K;
 };
 
-// Channels handled by one CTA of either scan kernel.
+// Channels handled by one CTA of the scan kernel.
 int channels_per_cta();
 
 // Device address of the library's error word on the current device (looked up once per device),
 // or null if the runtime fails.
 unsigned int* status_word();
 
-// The scan launches, one translation unit each: the fast kernel (bfloat16 io, delta as bfloat16
-// or int8 codes) and the precise kernel (fp32 io, or the exact ZOH).  phase1 = 1: segment
-// aggregates only (segments 0..S-2); phase1 = 0: the scan of all S segments.  With
-// prepare_only nothing is launched: only the kernel's shared-memory attribute is set.
-cudaError_t fast_launch_bf16(const ScanParams& p, int phase1, cudaStream_t stream, bool prepare_only);
-cudaError_t fast_launch_bf16_i8(const ScanParams& p, int phase1, cudaStream_t stream,
+// The scan launches, one translation unit per io type and delta storage (bfloat16 io with delta
+// as bfloat16 or int8 codes, fp32 io).  phase1 = 1: segment aggregates only (segments 0..S-2);
+// phase1 = 0: the scan of all S segments.  With prepare_only nothing is launched: only the
+// kernel's shared-memory attribute is set.
+cudaError_t scan_launch_f32(const ScanParams& p, int phase1, cudaStream_t stream, bool prepare_only);
+cudaError_t scan_launch_bf16(const ScanParams& p, int phase1, cudaStream_t stream, bool prepare_only);
+cudaError_t scan_launch_bf16_i8(const ScanParams& p, int phase1, cudaStream_t stream,
                                 bool prepare_only);
-cudaError_t precise_launch_f32(const ScanParams& p, int phase1, cudaStream_t stream,
-                               bool prepare_only);
-cudaError_t precise_launch_bf16(const ScanParams& p, int phase1, cudaStream_t stream,
-                                bool prepare_only);
-cudaError_t precise_launch_bf16_i8(const ScanParams& p, int phase1, cudaStream_t stream,
-                                   bool prepare_only);
-
-// Whether a call runs on the fast kernel (bfloat16 io without the exact ZOH) or the precise one.
-bool uses_fast_kernel(int io_dtype, bool zoh);
-
-// CTAs of a scan launch that one SM holds at once (the kernel's shared-memory and register
-// budget), for the automatic segment choice.
-int resident_ctas_per_sm(int io_dtype, bool zoh);
 
 // Everything a call needs before its first launch: the tensor maps of u, z and delta encoded into
 // p, and the shared-memory attributes of every kernel the call launches.  Nothing is launched,

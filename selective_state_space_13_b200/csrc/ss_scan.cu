@@ -4,7 +4,6 @@
 
 #include <mutex>
 
-#include "ss_fast.cuh"
 #include "ss_scan_kernels.cuh"
 
 namespace ss {
@@ -35,33 +34,21 @@ unsigned int* status_word()
 
 int channels_per_cta() { return 32 * kWarps; }
 
-bool uses_fast_kernel(int io_dtype, bool zoh) { return io_dtype == SS_BF16 && !zoh; }
-
-int resident_ctas_per_sm(int io_dtype, bool zoh)
-{
-    return uses_fast_kernel(io_dtype, zoh) ? fast::kMinBlocks : 6;
-}
-
 namespace {
 
 cudaError_t launch_any(const ScanParams& p, int io_dtype, int phase1, cudaStream_t stream,
                        bool prepare_only)
 {
-    const bool zoh = p.zoh != 0;
-    if (uses_fast_kernel(io_dtype, zoh))
-        return p.delta_scale ? fast_launch_bf16_i8(p, phase1, stream, prepare_only)
-                             : fast_launch_bf16(p, phase1, stream, prepare_only);
     if (io_dtype == SS_BF16)
-        return p.delta_scale ? precise_launch_bf16_i8(p, phase1, stream, prepare_only)
-                             : precise_launch_bf16(p, phase1, stream, prepare_only);
-    return precise_launch_f32(p, phase1, stream, prepare_only);
+        return p.delta_scale ? scan_launch_bf16_i8(p, phase1, stream, prepare_only)
+                             : scan_launch_bf16(p, phase1, stream, prepare_only);
+    return scan_launch_f32(p, phase1, stream, prepare_only);
 }
 
 }  // namespace
 
 cudaError_t prepare_scan(ScanParams& p, int io_dtype)
 {
-    static_assert(fast::kCh == 32 * kWarps, "both kernels read tiles of the same channel width");
     cudaError_t e;
     if (io_dtype == SS_BF16)
         e = p.delta_scale ? make_maps<__nv_bfloat16, int8_t>(p, p.z != nullptr, 32 * kWarps)
