@@ -190,20 +190,33 @@ class ClockSampler:
 
     def start(self):
         if self.ok:
+            # the sampler thread needs the interpreter lock every period: shorten the switch
+            # interval while it runs (the timed region of a small workload lasts milliseconds),
+            # and return once it is sampling
+            self._switch = sys.getswitchinterval()
+            sys.setswitchinterval(1e-4)
             self._thr = threading.Thread(target=self._run, daemon=True)
             self._thr.start()
+            t0 = time.time()
+            while not self.samples and time.time() - t0 < 1.0:
+                time.sleep(1e-4)
+            self._first = len(self.samples)
 
     def stop(self):
         if self._thr:
             self._stop.set()
             self._thr.join()
+            sys.setswitchinterval(self._switch)
 
     def report(self):
         if not self.ok:
             return None
-        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+        # the sample taken before the first step was enqueued is not part of the region
+        during = self.samples[getattr(self, "_first", 0):] or self.samples
+        return {"sm_mhz": statistics.median(during) if during else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
-                "samples": len(self.samples), "source": "NVML during the timed region"}
+                "samples": len(during), "period_ms": self.period * 1e3,
+                "source": "NVML during the timed region"}
 
 
 def workload_of(args) -> wl.Workload:
