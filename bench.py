@@ -45,6 +45,7 @@ METRIC = "selective-scan achieved HBM GB/s and % of peak; state-updates/s at 1 B
 UNIT = "GB/s"
 DEFAULT_WORKLOAD = "long"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 7700.0  # the specification figure, stated beside the measured peak
 FLUSH_BYTES = 256 << 20
 # FP32 operations of one state update in the form the kernels compute: the power-chain multiply
 # that gives exp(Delta*A[d,n]), the state multiply-add and the readout multiply-add
@@ -501,6 +502,14 @@ def run_ours(args):
                          "(%.3g state updates), timed %d times (%.1f s of CPU work)"
                          % (len(channels), w.dim, w.seqlen, w.K, w.updates() * frac, len(runs),
                             sum(runs))}
+        if threads > 1:
+            # the same oracle on one core, on a sample sized for a few seconds
+            ch1 = channels[:max(1, len(channels) * 2 // threads)]
+            s1 = time_oracle(inp, ch1, 1)
+            f1 = sample_fraction(w, ch1)
+            cpu["single_core"] = {"value": workload_bytes(w) * f1 / s1 / 1e9, "unit": UNIT,
+                                  "updates_per_s": w.updates() * f1 / s1, "seconds": s1,
+                                  "sample": "%d channels, all batch rows and steps" % len(ch1)}
 
     counters = {} if args.seqlen else recorded_counters(
         w.name + ("_conv%d" % w.conv if w.conv else "") + ("_int8" if w.delta_int8 else ""))
@@ -545,6 +554,8 @@ def run_ours(args):
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "peak_source": peak_src,
                      "algorithmic_bytes_per_launch": nbytes, "kernel_ms": kern_ms,
+                     "nominal": {"peak": NOMINAL_HBM_GBS, "frac": achieved / NOMINAL_HBM_GBS,
+                                 "source": "B200 HBM3e specification (HGX)"},
                      "alu": alu},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": sampler.report(),
