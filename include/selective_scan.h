@@ -51,8 +51,9 @@
  *   - The first selective_scan_fwd call on each device looks up the address of the library's
  *     device error word (cudaGetSymbolAddress, once); make that first call before capturing a
  *     stream into a CUDA graph.  The cached address (and the no-allocation scratch address of
- *     selective_scan_fwd_noalloc) belongs to the device's current context: after a
- *     cudaDeviceReset the library must not be called again in the same process.
+ *     selective_scan_fwd_noalloc, and the streams and events of selective_scan_fwd_host)
+ *     belongs to the device's current context: after a cudaDeviceReset the library must not be
+ *     called again in the same process.
  */
 #ifndef SELECTIVE_SCAN_H
 #define SELECTIVE_SCAN_H
