@@ -357,14 +357,11 @@ def run_ours(args):
         # this rank scans its slice of the one workload (batch rows or channels); the slices
         # are independent, so no data crosses between ranks
         from selective_state_space_13_b200 import shard
-        axis, lo, hi, w = shard.shard_workload(w_full, world, rank,
-                                               None if args.shard == "auto" else args.shard)
-        # every rank checks every slice, so all of them stop together (no collective waits)
-        empty = [r for r in range(world) if shard.shard_workload(w_full, world, r, axis)[2]
-                 <= shard.shard_workload(w_full, world, r, axis)[1]]
-        if empty:
-            raise SystemExit("--shard %s leaves rank(s) %s of %d without work; use fewer ranks"
-                             % (axis, empty, world))
+        try:
+            axis, lo, hi, w = shard.plan(w_full, world, rank,
+                                         None if args.shard == "auto" else args.shard)
+        except ValueError as e:  # raised on every rank alike: all stop together
+            raise SystemExit("--shard: %s; use fewer ranks" % e)
         inp = shard.shard_inputs(inp, axis, lo, hi)
         shard_info = {"axis": axis, "lo": lo, "hi": hi}
     t = wl.to_device(inp, device)

@@ -52,6 +52,17 @@ def shard_workload(w: wl.Workload, world: int, rank: int, axis: str | None = Non
     raise ValueError("axis must be 'batch' or 'channels'")
 
 
+def plan(w: wl.Workload, world: int, rank: int, axis: str | None = None):
+    """shard_workload for `rank`, after checking every rank's slice: a split that would leave a
+    rank without work raises ValueError on every rank alike (so all stop before any collective)."""
+    axis = axis or shard_axis(w, world)
+    empty = [r for r in range(world)
+             if (lambda s: s[2] <= s[1])(shard_workload(w, world, r, axis))]
+    if empty:
+        raise ValueError("splitting by %s leaves rank(s) %s of %d without work" % (axis, empty, world))
+    return shard_workload(w, world, rank, axis)
+
+
 def shard_inputs(inp: dict, axis: str, lo: int, hi: int) -> dict:
     """The inputs of one slice (arrays as make_inputs returns them), contiguous."""
     w = inp["workload"]

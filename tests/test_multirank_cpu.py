@@ -95,6 +95,32 @@ def test_slice_bounds_cover_every_unit_once():
         shard.slice_bounds(10, 2, 2)
 
 
+def test_shard_plans_of_the_workloads():
+    # the bench's split of each workload over 2, 4 and 8 ranks: by batch rows when there are
+    # enough, else by 64-channel tiles; a split that leaves a rank idle is refused for every rank
+    from selective_state_space_13_b200 import shard, workloads as wl
+    for name in ("m130", "long", "vim", "ss2d", "cromb"):
+        w = wl.WORKLOADS[name]
+        for world in (2, 4, 8):
+            axis = shard.shard_axis(w, world)
+            n = w.batch if axis == "batch" else w.dim
+            try:
+                parts = [shard.plan(w, world, r) for r in range(world)]
+            except ValueError:
+                # only a channel split can leave a rank idle (rows are split only when there
+                # are at least as many as ranks)
+                assert axis == "channels"
+                continue
+            assert sum(p[2] - p[1] for p in parts) == n
+            assert all(p[0] == axis and p[2] > p[1] for p in parts)
+    # long (one batch row) over 8 ranks: 640 channels each
+    parts = [shard.plan(wl.WORKLOADS["long"], 8, r) for r in range(8)]
+    assert {p[3].dim for p in parts} == {640}
+    # 192 channels cannot feed 8 ranks with whole 64-channel tiles
+    with pytest.raises(ValueError):
+        shard.plan(wl.variant("ss2d", batch=1), 8, 0)
+
+
 def _shard_worker(rank, world, port, q, axis):
     import datetime
 
