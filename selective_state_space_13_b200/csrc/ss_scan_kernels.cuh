@@ -350,8 +350,8 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
             mbar_arrive(&full[st]);
     };
 
-    // Convert tile `it`'s B (and C) to fp32 (producing warp).  On the fast path B carries the ln 2 of
-    // w = Delta*u / ln 2.
+    // Convert tile `it`'s B (and C) to the state type (producing warp).  On the fast path B
+    // carries the ln 2 of w = Delta*u / ln 2.
     auto convert = [&](int64_t it) {
         const int st = static_cast<int>(it % kStages);
         const int64_t t0 = t_begin + it * kTile;
