@@ -258,8 +258,11 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     }
 
     // B/C tiles are copied from a 16-byte aligned superset of their rows; `skip` is the offset
-    // (in elements) of the first wanted element inside the copied block.
-    auto bc_src = [&](const io_t* base, int64_t t0, int rows, uint32_t& bytes, int& skip) {
+    // (in elements) of the first wanted element inside the copied block.  With whole 16-byte
+    // rows (N * element size a multiple of 16) every tile starts aligned and `skip` is 0.
+    const bool bc_whole = (p.N * sizeof(io_t)) % 16 == 0;
+    auto bc_src = [&](const io_t* base, int64_t it, int rows, uint32_t& bytes, int& skip) {
+        const int64_t t0 = t_begin + it * kTile;
         const uintptr_t a0 = reinterpret_cast<uintptr_t>(base + (kb * p.L + t0) * p.N);
         const uintptr_t a1 = reinterpret_cast<uintptr_t>(base + (kb * p.L + t0 + rows) * p.N);
         const uintptr_t lo = a0 & ~static_cast<uintptr_t>(15);
@@ -285,15 +288,14 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     constexpr uint32_t kBox3 = static_cast<uint32_t>(DC) * 8 * sizeof(io_t);
     constexpr uint32_t kUZ = Lay::HAS_Z ? 2u : 1u;
 
-    // Fill the stage of time tile `it` (called by the producing warp).
-    auto issue = [&](int64_t it) {
-        const int st = static_cast<int>(it % kStages);
+    // Fill stage st with time tile `it` (called by the producing warp).
+    auto issue = [&](int64_t it, int st) {
         const int64_t t0 = t_begin + it * kTile;
         const int rows = tile_rows(it);
         uint32_t bbytes, cbytes = 0;
         int bskip, cskip;
-        const void* bsrc = bc_src(gB, t0, rows, bbytes, bskip);
-        const void* csrc = Lay::HAS_C ? bc_src(gC, t0, rows, cbytes, cskip) : nullptr;
+        const void* bsrc = bc_src(gB, it, rows, bbytes, bskip);
+        const void* csrc = Lay::HAS_C ? bc_src(gC, it, rows, cbytes, cskip) : nullptr;
         if (lane == 0) {
             uint32_t tx = kBoxDL + bbytes + cbytes;  // delta box, B, C
             if (umode == 0)
@@ -336,7 +338,8 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
         int32_t* orow = reinterpret_cast<int32_t*>(smem + Lay::OFF_OUT + st * Lay::OUT_STRIDE);
         for (int r = lane; r < rows; r += 32) {
             const int64_t pp = position(dir, p.L, p.H, p.W, t0 + r);
-            orow[r] = static_cast<int32_t>(pp * p.D);  // L * D < 2^31 (checked on the host)
+            // L * D < 2^31 (checked on the host): 32-bit arithmetic
+            orow[r] = static_cast<int32_t>(pp) * static_cast<int32_t>(p.D);
             if (umode == 2) {
                 bulk_g2s(smem + Lay::OFF_U + st * Lay::ROWS + r * Lay::ROW, gu + (ub * p.L + pp) * p.D + d0,
                          row_bytes, &full[st]);
@@ -352,15 +355,15 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
 
     // Convert tile `it`'s B (and C) to the state type (producing warp).  On the fast path B
     // carries the ln 2 of w = Delta*u / ln 2.
-    auto convert = [&](int64_t it) {
-        const int st = static_cast<int>(it % kStages);
-        const int64_t t0 = t_begin + it * kTile;
+    auto convert = [&](int64_t it, int st) {
         const int rows = tile_rows(it);
         uint32_t bytes;
         int bskip = 0, cskip = 0;
-        bc_src(gB, t0, rows, bytes, bskip);
-        if (Lay::HAS_C)
-            bc_src(gC, t0, rows, bytes, cskip);
+        if (!bc_whole) {
+            bc_src(gB, it, rows, bytes, bskip);
+            if (Lay::HAS_C)
+                bc_src(gC, it, rows, bytes, cskip);
+        }
         const io_t* br = reinterpret_cast<const io_t*>(smem + Lay::OFF_BR + st * Lay::BCRAW) + bskip;
         const io_t* cr = reinterpret_cast<const io_t*>(smem + Lay::OFF_CR + st * Lay::BCRAW) + cskip;
         st_t* bf = reinterpret_cast<st_t*>(smem + Lay::OFF_BF + st * Lay::BF_STRIDE);
@@ -518,22 +521,25 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
     if (warp == 0) {
         int64_t j = 0;
         for (; j < kStages - 2 && j < ntile_t; ++j)
-            issue(j);
+            issue(j, static_cast<int>(j));
         my_issued = j;
         if (lane == 0)
             *s_issued = static_cast<int>(j);
         if (!mbar_wait_bounded(&full[0], 0, kWaitLimitNs)) {
             failed = true;
         } else {
-            convert(0);
+            convert(0, 0);
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&ready[0]);
         }
     }
-    for (int64_t it = 0; it < ntile_t && !failed; ++it) {
-        const int st = static_cast<int>(it % kStages);
-        const uint32_t ph = static_cast<uint32_t>((it / kStages) & 1);
+    // stage st = it % kStages and phase parity ph = (it / kStages) & 1 of tile it, advanced at
+    // the end of each iteration (no 64-bit division per tile)
+    int st = 0;
+    uint32_t ph = 0;
+    for (int64_t it = 0; it < ntile_t && !failed;
+         ++it, ph ^= (st == kStages - 1) ? 1u : 0u, st = (st == kStages - 1) ? 0 : st + 1) {
         const int rows = tile_rows(it);
         if (*s_abort) {
             failed = true;
@@ -541,26 +547,29 @@ __global__ void __launch_bounds__(32 * WARPS, PHASE1 ? 8 : 6)
         }
         if (warp == static_cast<int>(it % WARPS)) {
             const int64_t n1 = it + 1;
+            // tile it+1: the next stage, in the next phase when it wraps
+            const int st1 = (st == kStages - 1) ? 0 : st + 1;
+            const uint32_t ph1 = ph ^ ((st == kStages - 1) ? 1u : 0u);
             if (n1 < ntile_t) {
-                if (!mbar_wait_bounded(&full[n1 % kStages],
-                                       static_cast<uint32_t>((n1 / kStages) & 1), kWaitLimitNs)) {
+                if (!mbar_wait_bounded(&full[st1], ph1, kWaitLimitNs)) {
                     failed = true;
                 } else {
-                    convert(n1);
+                    convert(n1, st1);
                     __syncwarp();
                     if (lane == 0)
-                        mbar_arrive(&ready[n1 % kStages]);
+                        mbar_arrive(&ready[st1]);
                 }
             }
+            // tile it+kStages-2 goes to the stage tile it-2 used; that stage's previous phase
+            // (the release by tile it-2) has parity ((it + kStages - 2) / kStages - 1) & 1
             const int64_t nx = it + kStages - 2;
+            const int stx = (st >= 2) ? st - 2 : st + kStages - 2;
+            const uint32_t phx = ph ^ ((st >= 2) ? 1u : 0u) ^ 1u;
             if (!failed && nx < ntile_t) {
-                if (nx >= kStages &&
-                    !mbar_wait_bounded(&empty[nx % kStages],
-                                       static_cast<uint32_t>(((nx / kStages) - 1) & 1),
-                                       kWaitLimitNs)) {
+                if (nx >= kStages && !mbar_wait_bounded(&empty[stx], phx, kWaitLimitNs)) {
                     failed = true;
                 } else {
-                    issue(nx);
+                    issue(nx, stx);
                     my_issued = nx + 1;
                     if (lane == 0)
                         *s_issued = static_cast<int>(nx + 1);
